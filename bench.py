@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 int4 MoE layer (libmoe), one JSON line on stdout (rank 0).
+
+Headline workload (default): the 16384-token prefill of a 40-layer stack, processed as four
+4096-token chunks per layer (chunk-major: each chunk passes through layers 0..39), Zipf(1.2)
+routing skew, synthetic random-init weights of the 256-expert int4 layer.  value = MoE-layer
+tokens/s = tokens x layers / step time.  A second measurement on the same line ("decode") times
+batch-1 decode over 40 distinct layers replayed as one CUDA graph (us per token per layer).
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the launching stream,
+bracketed by a barrier + synchronize, max over ranks.  Every layer's weights (457 MB) exceed the
+126 MB L2, so no flush is needed between steps.  Per-kernel durations for the roofline come from
+events the library records around each of its launches in a separate profiled pass of K steps.
+
+Multi-GPU (torchrun): every rank runs its own replica on its own tokens (the layer shards by
+tokens with no exchange), value = all ranks' tokens / max-over-ranks time ("scaling": "weak").
+
+--impl reference: the CPU oracle (test infrastructure) timed as it stands on the host cores over a
+bounded token sample of the same workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill16k_zipf",
+                    choices=["prefill16k_zipf", "prefill4k_zipf", "prefill512", "decode"])
+    ap.add_argument("--layers", type=int, default=None, help="override the stack depth (quick runs)")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle sample time")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------ dist
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend):
+        import torch
+        import torch.distributed as dist
+        if self.world > 1:
+            import datetime
+            kw = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        dev = torch.device("cuda", self.local) if torch.cuda.is_available() else torch.device("cpu")
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [v.strip() for v in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = max((num(r[2]) for r in rows if num(r[2]) is not None), default=None)
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        # "under load": samples drawing more than idle power
+        loaded = [s for s, pw in zip(sm, power) if pw is not None and pw > 250] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------------------------------- stacks
+def build_stack(shape, n_layers, max_tokens, decode_max_tokens, keep_host_layer0=False):
+    import torch
+    from bit_grouped_expert_router_b200 import _lib as M
+    from bit_grouped_expert_router_b200 import synth
+    layers, host0 = [], None
+    for l in range(n_layers):
+        w = synth.make_layer(shape, l, device="cuda")
+        if l == 0 and keep_host_layer0:
+            host0 = {k: (v.cpu() if v is not None else None) for k, v in w.items()}
+        layers.append(M.Layer.from_shape(w, shape, max_tokens=max_tokens, decode_max_tokens=decode_max_tokens))
+        del w
+    torch.cuda.synchronize()
+    return layers, host0
+
+
+def timed(fn, steps, warmup, dist):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = e0.elapsed_time(e1) / steps
+    return dist.max(ms)
+
+
+def profile_pass(layers, fn, steps):
+    import torch
+    for L in layers:
+        L.profile(True)
+    for _ in range(steps):
+        fn()
+    torch.cuda.synchronize()
+    tot = {}
+    for L in layers:
+        for k, (ms, n) in L.profile_read().items():
+            a = tot.setdefault(k, [0.0, 0])
+            a[0] += ms
+            a[1] += n
+        L.profile(False)
+    return {k: {"avg_us": 1000.0 * v[0] / v[1], "launches": v[1], "total_ms": v[0]} for k, v in tot.items()}
+
+
+# ---------------------------------------------------------------------------------------- prefill
+def gemm_flops(shape):
+    rows = shape.T * shape.k + (shape.T if shape.has_shared else 0)
+    return 2.0 * rows * 2 * shape.I * shape.H, 2.0 * rows * shape.I * shape.H
+
+
+def run_prefill(args, dist, peaks, peak_src):
+    import torch
+    from bit_grouped_expert_router_b200 import synth
+    shape = synth.WORKLOADS[args.workload]
+    n_layers = args.layers or shape.layers
+    chunks = shape.chunks
+    layers, host0 = build_stack(shape, n_layers, shape.T, 16, keep_host_layer0=True)
+    xs = [[synth.make_x(shape, l, c, device="cuda") for c in range(chunks)] for l in range(n_layers)]
+    out = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        for c in range(chunks):
+            for l in range(n_layers):
+                layers[l].forward(xs[l][c], out=out)
+
+    tokens_per_step = shape.T * chunks * n_layers  # layer-tokens
+    clocks = ClockSampler(torch.cuda.current_device())
+    # warm-up outside the sampled window, then the timed region with clocks sampled
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks.start()
+    ms = timed(step, args.steps, 0, dist)
+    clk = clocks.stop()
+    for L in layers:
+        assert L.status() == 0, "device status after the timed region"
+    value = dist.world * tokens_per_step / (ms / 1000.0)
+
+    prof = profile_pass(layers, step, args.steps)
+    f_gu, f_dn = gemm_flops(shape)
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])  # fp16 dense == bf16 dense
+    roof = None
+    if "gemm_gateup" in prof:
+        a = f_gu / (prof["gemm_gateup"]["avg_us"] * 1e-6) / 1e12
+        roof = {"bound": "tensor", "kernel": "gemm_gateup (tcgen05 grouped GEMM + SwiGLU)",
+                "achieved": round(a, 1), "peak": peak_tf, "unit": "TFLOP/s", "frac": round(a / peak_tf, 4),
+                "traffic": None, "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16 dense rate)",
+                "flops_per_launch": f_gu}
+    gg = None
+    if "gemm_gateup" in prof and "gemm_down" in prof:
+        t = (prof["gemm_gateup"]["avg_us"] + prof["gemm_down"]["avg_us"]) * 1e-6
+        a = (f_gu + f_dn) / t / 1e12
+        gg = {"achieved_tflops": round(a, 1), "frac_of_peak": round(a / peak_tf, 4),
+              "us_per_chunk": round(t * 1e6, 1)}
+    res = dict(value=value, ms=ms, clocks=clk, roofline=roof, kernels=prof, grouped_gemm=gg,
+               launches=7 * chunks * n_layers * args.steps, shape=shape, n_layers=n_layers,
+               tokens_per_step=tokens_per_step)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    if not args.no_e2e:
+        xh = [[xs[l][c].cpu().pin_memory() for c in range(chunks)] for l in range(n_layers)]
+        oh = torch.empty((shape.T, shape.H), dtype=torch.bfloat16).pin_memory()
+
+        def step_host():
+            for c in range(chunks):
+                for l in range(n_layers):
+                    layers[l].forward_host(xh[l][c], oh)
+        ms_e2e = timed(step_host, max(1, args.steps // 2), 1, dist)
+        bytes_io = shape.T * shape.H * 2 * chunks * n_layers
+        res["e2e"] = {"value": dist.world * tokens_per_step / (ms_e2e / 1000.0), "unit": "tokens/s",
+                      "h2d_bytes_per_step": bytes_io, "d2h_bytes_per_step": bytes_io,
+                      "ms_per_step": round(ms_e2e, 3), "api": "moe_forward_host (pinned host buffers)"}
+        del xh
+    res["host0"] = host0
+    res["x0"] = xs[0][0].cpu()
+    for L in layers:
+        L.close()
+    del xs
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode(args, dist, peaks, peak_src):
+    import torch
+    from bit_grouped_expert_router_b200 import synth
+    shape = synth.WORKLOADS["decode"]
+    n_layers = args.layers or shape.layers
+    layers, _ = build_stack(shape, n_layers, 16, 16)
+    xs = [synth.make_x(shape, l, 0, device="cuda") for l in range(n_layers)]
+    outs = [torch.empty((1, shape.H), dtype=torch.bfloat16, device="cuda") for _ in range(n_layers)]
+
+    def eager():
+        for l in range(n_layers):
+            layers[l].forward(xs[l], out=outs[l])
+
+    eager()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        eager()
+    torch.cuda.synchronize()
+    ms = timed(g.replay, max(args.steps, 20) * 5, args.warmup, dist)
+    us_layer = ms * 1000.0 / n_layers
+    prof = profile_pass(layers, eager, max(args.steps, 20))
+    expert_bytes = (shape.I // 64) * (shape.H // 64) * 4608 + (shape.H // 128) * (shape.I // 64) * 4608
+    nexp = shape.k + 1
+    hbm = peaks["hbm_gbs"]
+    roof = None
+    if "gemv_gateup" in prof and "gemv_down" in prof:
+        b_gu = nexp * (shape.I // 64) * (shape.H // 64) * 4608 + shape.H * 2
+        b_dn = nexp * (shape.H // 128) * (shape.I // 64) * 4608 + shape.H * 2
+        t = (prof["gemv_gateup"]["avg_us"] + prof["gemv_down"]["avg_us"]) * 1e-6
+        a = (b_gu + b_dn) / t / 1e9
+        roof = {"bound": "hbm", "kernel": "sparse GEMV gate/up + down (eager, profiled)",
+                "achieved": round(a, 1), "peak": hbm, "unit": "GB/s", "frac": round(a / hbm, 4),
+                "traffic": None, "bytes_per_token": b_gu + b_dn,
+                "peak_source": f"{peak_src} hbm_gbs"}
+    layer_bytes = nexp * expert_bytes + shape.E * shape.H * 4 + shape.H * 4 + 2 * shape.H * 2
+    for L in layers:
+        assert L.status() == 0
+        L.close()
+    del g
+    return {"metric": "MoE-layer decode us/token/layer (batch 1, 40 distinct layers, one CUDA graph)",
+            "value": round(us_layer, 3), "unit": "us/token/layer", "higher_is_better": False,
+            "whole_layer_hbm_frac": round(layer_bytes / (us_layer * 1e-6) / 1e9 / hbm, 4),
+            "whole_layer_bytes": layer_bytes, "roofline": roof, "kernels": prof,
+            "gpu_launches_per_step": 4 * n_layers}
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+def cpu_baseline(host0, x0, shape, target_s):
+    import oracle
+    ol = oracle.OracleLayer.from_shape(host0, shape)
+    n = 8
+    t0 = time.perf_counter()
+    ol.forward(x0, tokens=list(range(n)))
+    dt = time.perf_counter() - t0
+    n2 = int(min(shape.T - n, max(8, (target_s - dt) / max(dt / n, 1e-6))))
+    t1 = time.perf_counter()
+    if n2 > 0:
+        ol.forward(x0, tokens=list(range(n, n + n2)))
+    dt2 = time.perf_counter() - t1
+    total_n, total_t = (n + n2, dt + dt2)
+    return {"value": round(total_n / total_t, 3), "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{total_n} tokens of layer 0, chunk 0 through one MoE layer (fp64 oracle, "
+                      f"{total_t:.1f} s); per-layer tokens/s comparable to value"}
+
+
+def run_reference(args, dist):
+    """The oracle as the reference arm: rank 0 only, bounded token sample per step."""
+    if dist.rank != 0:
+        return
+    import torch
+    import oracle
+    from bit_grouped_expert_router_b200 import synth
+    shape = synth.WORKLOADS[args.workload]
+    w = synth.make_layer(shape, 0)
+    x = synth.make_x(shape, 0, 0)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    per_step = 8 if shape.T > 1 else 1
+    t_tok = []
+    for i in range(args.warmup + args.steps):
+        tok = [(i * per_step + j) % shape.T for j in range(per_step)]
+        t0 = time.perf_counter()
+        ol.forward(x, tokens=tok)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            t_tok.append(dt)
+    ms = 1000.0 * sum(t_tok) / len(t_tok)
+    if args.workload == "decode":
+        value, unit, hib, metric = ms * 1000.0 / per_step, "us/token/layer", False, \
+            "MoE-layer decode us/token/layer"
+    else:
+        value, unit, hib, metric = per_step / (ms / 1000.0), "tokens/s", True, "MoE-layer prefill tokens/s"
+    sample = f"{per_step} tokens of layer 0 per step through one MoE layer (fp64 CPU oracle)"
+    line = {"impl": "reference", "metric": metric, "value": round(value, 4), "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": hib,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "T": shape.T, "H": shape.H, "E": shape.E, "k": shape.k,
+                       "I": shape.I, "layers_sampled": 1},
+            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    import torch
+    dist.init("nccl")
+    torch.cuda.set_device(dist.local)
+    peaks, peak_src = load_peaks()
+    from bit_grouped_expert_router_b200 import build as B
+    B.build()
+
+    line = None
+    if args.workload == "decode":
+        d = run_decode(args, dist, peaks, peak_src)
+        line = {"metric": d["metric"], "value": d["value"] / dist.world, "unit": d["unit"],
+                "higher_is_better": False, "roofline": d["roofline"], "decode_detail": d}
+    else:
+        r = run_prefill(args, dist, peaks, peak_src)
+        shape = r["shape"]
+        line = {"metric": f"MoE-layer prefill tokens/s ({shape.T * shape.chunks}-token prompt in "
+                          f"{shape.T}-token chunks, {r['n_layers']} layers; also decode us/token/layer)",
+                "value": round(r["value"], 1), "unit": "tokens/s", "higher_is_better": True,
+                "ms_per_step": round(r["ms"], 3), "roofline": r["roofline"], "grouped_gemm": r["grouped_gemm"],
+                "kernels": r["kernels"], "gpu_launches": r["launches"], "clocks": r["clocks"]}
+        if "e2e" in r:
+            line["e2e"] = r["e2e"]
+        if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(r["host0"], r["x0"], shape, args.cpu_seconds)
+        if not args.no_decode:
+            d = run_decode(args, dist, peaks, peak_src)
+            line["decode"] = d
+        line["config"] = {"workload": args.workload, "tokens": shape.T * shape.chunks, "chunk": shape.T,
+                          "layers": r["n_layers"], "H": shape.H, "I": shape.I, "E": shape.E, "k": shape.k,
+                          "shared_expert": shape.has_shared, "zipf_s": shape.zipf_s,
+                          "weights": "int4 g64 asymmetric, bf16 scale/bias (repacked fp16)",
+                          "l2": "inputs larger than L2: 457 MB of weights per layer, 40 distinct layers",
+                          "decode_workload": "decode (T=1, 40 layers, CUDA graph)"}
+    base = {"n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp16", "data": "synthetic (seeded random-init weights and activations)"}
+    for k, v in base.items():
+        line.setdefault(k, v)
+    line.setdefault("gpu_launches", None)
+    if dist.rank == 0:
+        print(json.dumps(line, default=str), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

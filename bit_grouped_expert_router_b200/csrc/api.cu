@@ -1,0 +1,552 @@
+// api.cu -- the C ABI (include/moe.h): handle lifetime, workspace, tensor maps and the launch
+// sequence of one forward call.  Host code only; every step of the layer runs in the kernels.
+//
+// Prefill path (T > decode_max_tokens), all stream-ordered, no host synchronisation:
+//   router logits -> top-k/gates/histogram -> bucket scan + tile list -> scatter (bucketed fp16
+//   rows, zeroed accumulator) -> tcgen05 gate/up GEMM + SwiGLU -> tcgen05 down GEMM + combine
+//   -> bf16 finalize.
+// Decode path (T <= decode_max_tokens): split-K router -> top-k/gates -> sparse GEMV gate/up +
+//   SwiGLU -> sparse GEMV down + gated combine (bf16 out).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+#define CUDA_TRY(expr)                                                                              \
+    do {                                                                                            \
+        cudaError_t _e = (expr);                                                                    \
+        if (_e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(_e)); \
+    } while (0)
+
+struct DeviceGuard {
+    int prev = -1;
+    bool changed = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+            changed = cudaSetDevice(dev) == cudaSuccess;
+        }
+    }
+    ~DeviceGuard() {
+        if (changed) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Sizes derived from a configuration.
+struct Layout {
+    int H, I, E, k, G, Tm, Tdec, ks_dec, nblk_max, max_tiles, rows_cap;
+    size_t w_gu_bytes, w_dn_bytes, router_bytes, weights_bytes;
+    // workspace offsets
+    size_t o_part, o_idx, o_gates, o_sg, o_hist, o_counts, o_offsets, o_tiles, o_ntiles, o_perm, o_rtok,
+        o_rgate, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_counters, o_stage_x, o_stage_out, ws_bytes;
+};
+
+Layout make_layout(const moe_config& c) {
+    Layout L{};
+    L.H = c.hidden;
+    L.I = c.inter;
+    L.E = c.num_experts;
+    L.k = c.top_k;
+    L.G = c.num_experts + (c.has_shared ? 1 : 0);
+    L.Tm = c.max_tokens;
+    L.Tdec = c.decode_max_tokens < c.max_tokens ? (c.decode_max_tokens > 0 ? c.decode_max_tokens : 0)
+                                                 : c.max_tokens;
+    L.ks_dec = c.hidden / kRouterKSlice;
+    L.nblk_max = (L.Tm + kTokPerBucketBlk - 1) / kTokPerBucketBlk;
+    L.rows_cap = L.Tm * L.k + (c.has_shared ? L.Tm : 0);
+    L.max_tiles = (L.rows_cap + kBN - 1) / kBN + L.G;
+    const size_t per_mat_gu = (size_t)(L.I / 64) * (L.H / 64) * kBlockBytes;   // gate+up rows 2I
+    const size_t per_mat_dn = (size_t)(L.H / 128) * (L.I / 64) * kBlockBytes;
+    L.w_gu_bytes = per_mat_gu * L.G;
+    L.w_dn_bytes = per_mat_dn * L.G;
+    L.router_bytes = sizeof(float) * ((size_t)L.H * L.E + L.E + L.H);
+    L.weights_bytes = align_up(L.w_gu_bytes, 256) + align_up(L.w_dn_bytes, 256) + align_up(L.router_bytes, 256);
+
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes, 256);
+        return at;
+    };
+    const size_t part_rows = std::max((size_t)L.Tm, (size_t)L.ks_dec * (size_t)L.Tdec);
+    L.o_part = take(sizeof(float) * part_rows * L.E);
+    L.o_idx = take(sizeof(int) * (size_t)L.Tm * L.k);
+    L.o_gates = take(sizeof(float) * (size_t)L.Tm * L.k);
+    L.o_sg = take(sizeof(float) * (size_t)L.Tm);
+    L.o_hist = take(sizeof(int) * (size_t)L.nblk_max * L.E);
+    L.o_counts = take(sizeof(int) * (size_t)(L.G + 1));
+    L.o_offsets = take(sizeof(int) * (size_t)(L.G + 2));
+    L.o_tiles = take(sizeof(int4) * (size_t)L.max_tiles);
+    L.o_ntiles = take(sizeof(int) * 4);
+    L.o_perm = take(sizeof(int) * (size_t)L.Tm * L.k);
+    L.o_rtok = take(sizeof(int) * (size_t)L.rows_cap);
+    L.o_rgate = take(sizeof(float) * (size_t)L.rows_cap);
+    L.o_xp = take(sizeof(__half) * (size_t)L.rows_cap * L.H);
+    L.o_act = take(sizeof(__half) * (size_t)L.rows_cap * L.I);
+    L.o_acc = take(sizeof(float) * (size_t)L.Tm * L.H);
+    L.o_dact = take(sizeof(float) * (size_t)std::max(L.Tdec, 1) * (L.k + 1) * L.I);
+    L.o_dscale = take(sizeof(float) * 2 * (size_t)std::max(L.Tdec, 1) * (L.k + 1) * (L.I / 64));
+    L.o_status = take(sizeof(uint32_t) * 4);
+    L.o_counters = take(sizeof(unsigned) * 64);
+    L.o_stage_x = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
+    L.o_stage_out = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
+    L.ws_bytes = o;
+    return L;
+}
+
+int validate_config(const moe_config* c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+    if (c->group != 64) return fail(MOE_ERR_INVALID_ARG, "group must be 64 (got %d)", c->group);
+    if (c->hidden <= 0 || c->hidden % 128 != 0) return fail(MOE_ERR_INVALID_ARG, "hidden must be a positive multiple of 128");
+    if (c->inter <= 0 || c->inter % 64 != 0) return fail(MOE_ERR_INVALID_ARG, "inter must be a positive multiple of 64");
+    if (c->num_experts < 1 || c->num_experts > 256) return fail(MOE_ERR_INVALID_ARG, "num_experts must be in [1, 256]");
+    if (c->top_k < 1 || c->top_k > c->num_experts || c->top_k > 32)
+        return fail(MOE_ERR_INVALID_ARG, "top_k must be in [1, min(num_experts, 32)]");
+    if (c->has_shared != 0 && c->has_shared != 1) return fail(MOE_ERR_INVALID_ARG, "has_shared must be 0 or 1");
+    if (c->max_tokens < 1 || c->max_tokens > 65536) return fail(MOE_ERR_INVALID_ARG, "max_tokens must be in [1, 65536]");
+    if (c->decode_max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "decode_max_tokens must be >= 0");
+    if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_TEST_STALL))
+        return fail(MOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
+    return MOE_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D fp16 row-major [rows, cols] tensor, box {64 columns, box_rows rows}, 128-byte swizzle.
+int encode_rows_map(CUtensorMap* m, void* base, int rows, int cols, int box_rows) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return MOE_OK;
+}
+
+}  // namespace
+
+constexpr int kProfCalls = 1024;
+constexpr int kProfEvents = 8;  // at most 7 kernels per call + the leading event
+
+struct moe_handle {
+    int device = 0;
+    // per-kernel profiling (moe_profile_enable)
+    bool prof = false;
+    cudaEvent_t* prof_ev = nullptr;        // [kProfCalls][kProfEvents]
+    int prof_slot[kProfCalls][kProfEvents] = {};
+    int prof_nev[kProfCalls] = {};
+    int prof_calls = 0;
+    moe_config cfg{};
+    Layout L{};
+    int num_sms = 0;
+    uint8_t* wbuf = nullptr;
+    uint8_t* ws = nullptr;
+    Ctx base{};
+    CUtensorMap tm_xp{}, tm_act{};
+    cudaStream_t last_stream = nullptr;
+    bool inexact_scales = false;
+};
+
+namespace {
+
+Ctx make_ctx(const moe_handle* h, int T, const uint16_t* x, uint16_t* out, bool decode) {
+    Ctx c = h->base;
+    c.T = T;
+    c.x = x;
+    c.out = out;
+    c.nblk = (T + kTokPerBucketBlk - 1) / kTokPerBucketBlk;
+    c.ks = decode ? h->L.ks_dec : 1;
+    return c;
+}
+
+int check_call(moe_handle* h, const void* x, int32_t T, const void* out, bool need_out) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+    if (T > h->cfg.max_tokens) return fail(MOE_ERR_TOO_LARGE, "T = %d exceeds max_tokens = %d", T, h->cfg.max_tokens);
+    if (T > 0 && (!x || !aligned16(x))) return fail(MOE_ERR_INVALID_ARG, "x must be a 16-byte aligned device pointer");
+    if (T > 0 && need_out && (!out || !aligned16(out)))
+        return fail(MOE_ERR_INVALID_ARG, "out must be a 16-byte aligned device pointer");
+    return MOE_OK;
+}
+
+bool use_decode(const moe_handle* h, int T) { return T <= h->cfg.decode_max_tokens; }
+
+// Profiling: one event before the first kernel of a call and one after each kernel.
+struct Prof {
+    moe_handle* h;
+    cudaStream_t st;
+    int call = -1;
+    Prof(moe_handle* hh, cudaStream_t s) : h(hh), st(s) {
+        if (h->prof && h->prof_calls < kProfCalls) {
+            call = h->prof_calls++;
+            h->prof_nev[call] = 0;
+            mark(-1);
+        }
+    }
+    void mark(int slot) {
+        if (call < 0) return;
+        const int n = h->prof_nev[call];
+        if (n >= kProfEvents) return;
+        cudaEventRecord(h->prof_ev[call * kProfEvents + n], st);
+        h->prof_slot[call][n] = slot;
+        h->prof_nev[call] = n + 1;
+    }
+};
+
+int enqueue_routing(Prof& pf, const Ctx& c, bool decode, cudaStream_t st) {
+    CUDA_TRY(launch_router_simt(c, st));
+    pf.mark(0);
+    CUDA_TRY(launch_topk(c, !decode, st));
+    pf.mark(1);
+    if (!decode) {
+        CUDA_TRY(launch_bucket_scan(c, st));
+        pf.mark(2);
+        CUDA_TRY(launch_scatter(c, st));
+        pf.mark(3);
+    }
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_version(void) { return 10000; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+size_t moe_device_bytes(const moe_config* cfg) {
+    if (validate_config(cfg) != MOE_OK) return 0;
+    const Layout L = make_layout(*cfg);
+    return L.weights_bytes + L.ws_bytes;
+}
+
+int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* stream, moe_handle** out) {
+    g_last_error.clear();
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    int rc = validate_config(cfg);
+    if (rc != MOE_OK) return rc;
+    if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
+    const void* req[] = {w->q_gate, w->q_up, w->q_down, w->s_gate, w->b_gate, w->s_up, w->b_up, w->s_down, w->b_down,
+                         w->router};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "a required weight pointer is NULL or misaligned");
+    if (cfg->has_shared) {
+        const void* sh[] = {w->qs_gate, w->qs_up, w->qs_down, w->ss_gate, w->bs_gate, w->ss_up, w->bs_up,
+                            w->ss_down, w->bs_down, w->shared_gate};
+        for (const void* p : sh)
+            if (!p || !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "a shared-expert pointer is NULL or misaligned");
+    }
+    if (w->router_bias && !aligned16(w->router_bias)) return fail(MOE_ERR_INVALID_ARG, "router_bias misaligned");
+
+    int ndev = 0;
+    CUDA_TRY(cudaGetDeviceCount(&ndev));
+    if (device < 0 || device >= ndev) return fail(MOE_ERR_INVALID_ARG, "device %d out of range", device);
+    cudaDeviceProp prop;
+    CUDA_TRY(cudaGetDeviceProperties(&prop, device));
+    if (prop.major != 10 || prop.minor != 0)
+        return fail(MOE_ERR_UNSUPPORTED_DEVICE, "device %d is sm_%d%d; libmoe needs sm_100 (B200)", device, prop.major,
+                    prop.minor);
+    DeviceGuard guard(device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    moe_handle* h = new moe_handle();
+    h->device = device;
+    h->cfg = *cfg;
+    h->L = make_layout(*cfg);
+    h->num_sms = prop.multiProcessorCount;
+    const Layout& L = h->L;
+    auto cleanup = [&](int code) {
+        if (h->wbuf) cudaFree(h->wbuf);
+        if (h->ws) cudaFree(h->ws);
+        delete h;
+        return code;
+    };
+    cudaError_t e = cudaMalloc(&h->wbuf, L.weights_bytes);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMalloc(weights %zu B): %s", L.weights_bytes, cudaGetErrorString(e)));
+    e = cudaMalloc(&h->ws, L.ws_bytes);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMalloc(workspace %zu B): %s", L.ws_bytes, cudaGetErrorString(e)));
+    e = cudaMemsetAsync(h->ws, 0, L.ws_bytes, st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e)));
+
+    uint8_t* w_gu = h->wbuf;
+    uint8_t* w_dn = w_gu + align_up(L.w_gu_bytes, 256);
+    float* wrt = reinterpret_cast<float*>(w_dn + align_up(L.w_dn_bytes, 256));
+    float* rbias = wrt + (size_t)L.H * L.E;
+    float* sgw = rbias + L.E;
+    uint32_t* status = reinterpret_cast<uint32_t*>(h->ws + L.o_status);
+
+    RepackArgs a{};
+    a.E = L.E;
+    a.inexact = status + 1;
+    a.gateup = 1;
+    a.rows_per_mat = L.I;
+    a.cols = L.H;
+    a.q[0] = w->q_gate; a.s[0] = w->s_gate; a.b[0] = w->b_gate;
+    a.q[1] = w->q_up;   a.s[1] = w->s_up;   a.b[1] = w->b_up;
+    a.qs[0] = w->qs_gate; a.ss[0] = w->ss_gate; a.bs[0] = w->bs_gate;
+    a.qs[1] = w->qs_up;   a.ss[1] = w->ss_up;   a.bs[1] = w->bs_up;
+    a.dst = w_gu;
+    e = launch_repack(a, L.G, L.I / 64, L.H / 64, st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "repack gate/up: %s", cudaGetErrorString(e)));
+    RepackArgs d{};
+    d.E = L.E;
+    d.inexact = status + 1;
+    d.gateup = 0;
+    d.rows_per_mat = L.H;
+    d.cols = L.I;
+    d.q[0] = w->q_down; d.s[0] = w->s_down; d.b[0] = w->b_down;
+    d.q[1] = w->q_down; d.s[1] = w->s_down; d.b[1] = w->b_down;
+    d.qs[0] = w->qs_down; d.ss[0] = w->ss_down; d.bs[0] = w->bs_down;
+    d.qs[1] = w->qs_down; d.ss[1] = w->ss_down; d.bs[1] = w->bs_down;
+    d.dst = w_dn;
+    e = launch_repack(d, L.G, L.H / 128, L.I / 64, st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "repack down: %s", cudaGetErrorString(e)));
+    e = launch_router_prep(w->router, w->router_bias, cfg->has_shared ? w->shared_gate : nullptr, L.H, L.E, wrt, rbias,
+                           sgw, st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router prep: %s", cudaGetErrorString(e)));
+    uint32_t flags_host[2] = {0, 0};
+    e = cudaMemcpyAsync(flags_host, status, sizeof flags_host, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "create: %s", cudaGetErrorString(e)));
+    h->inexact_scales = flags_host[1] != 0;
+    e = cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "create: %s", cudaGetErrorString(e)));
+
+    Ctx& c = h->base;
+    c.H = L.H; c.I = L.I; c.E = L.E; c.k = L.k; c.G = L.G; c.has_shared = cfg->has_shared;
+    c.max_tiles = L.max_tiles;
+    c.rows_cap = L.rows_cap;
+    c.flags = cfg->flags;
+    c.w_gu = w_gu; c.w_dn = w_dn; c.wrt = wrt; c.rbias = rbias; c.sgw = sgw;
+    uint8_t* ws = h->ws;
+    c.part = reinterpret_cast<float*>(ws + L.o_part);
+    c.idx = reinterpret_cast<int*>(ws + L.o_idx);
+    c.gates = reinterpret_cast<float*>(ws + L.o_gates);
+    c.sg = reinterpret_cast<float*>(ws + L.o_sg);
+    c.hist = reinterpret_cast<int*>(ws + L.o_hist);
+    c.counts = reinterpret_cast<int*>(ws + L.o_counts);
+    c.offsets = reinterpret_cast<int*>(ws + L.o_offsets);
+    c.tiles1 = reinterpret_cast<int4*>(ws + L.o_tiles);
+    c.tiles2 = c.tiles1;
+    c.ntiles = reinterpret_cast<int*>(ws + L.o_ntiles);
+    c.perm = reinterpret_cast<int*>(ws + L.o_perm);
+    c.row_token = reinterpret_cast<int*>(ws + L.o_rtok);
+    c.row_gate = reinterpret_cast<float*>(ws + L.o_rgate);
+    c.xp = reinterpret_cast<__half*>(ws + L.o_xp);
+    c.act = reinterpret_cast<__half*>(ws + L.o_act);
+    c.acc = reinterpret_cast<float*>(ws + L.o_acc);
+    c.dact = reinterpret_cast<float*>(ws + L.o_dact);
+    c.dscale = reinterpret_cast<float*>(ws + L.o_dscale);
+    c.status = status;
+    c.counters = reinterpret_cast<unsigned*>(ws + L.o_counters);
+
+    rc = encode_rows_map(&h->tm_xp, c.xp, L.rows_cap, L.H, kBN);
+    if (rc == MOE_OK) rc = encode_rows_map(&h->tm_act, c.act, L.rows_cap, L.I, kBN);
+    if (rc != MOE_OK) return cleanup(rc);
+    h->last_stream = st;
+    *out = h;
+    return MOE_OK;
+}
+
+int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void* stream) {
+    int rc = check_call(h, x, T, out, true);
+    if (rc != MOE_OK || T == 0) return rc;
+    DeviceGuard guard(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    const bool decode = use_decode(h, T);
+    const Ctx c = make_ctx(h, T, x, out, decode);
+    Prof pf(h, st);
+    rc = enqueue_routing(pf, c, decode, st);
+    if (rc != MOE_OK) return rc;
+    if (decode) {
+        CUDA_TRY(launch_gemv_gateup(c, st));
+        pf.mark(7);
+        CUDA_TRY(launch_gemv_down(c, st));
+        pf.mark(8);
+    } else {
+        CUDA_TRY(launch_gemm_gateup(c, h->tm_xp, h->num_sms, st));
+        pf.mark(4);
+        CUDA_TRY(launch_gemm_down(c, h->tm_act, h->num_sms, st));
+        pf.mark(5);
+        CUDA_TRY(launch_finalize(c, st));
+        pf.mark(6);
+    }
+    return MOE_OK;
+}
+
+int moe_forward_host(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t* out_host, void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+    if (T > h->cfg.max_tokens) return fail(MOE_ERR_TOO_LARGE, "T = %d exceeds max_tokens = %d", T, h->cfg.max_tokens);
+    if (T == 0) return MOE_OK;
+    if (!x_host || !out_host) return fail(MOE_ERR_INVALID_ARG, "host buffers must not be NULL");
+    DeviceGuard guard(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint16_t* dx = reinterpret_cast<uint16_t*>(h->ws + h->L.o_stage_x);
+    uint16_t* dout = reinterpret_cast<uint16_t*>(h->ws + h->L.o_stage_out);
+    const size_t bytes = sizeof(uint16_t) * (size_t)T * h->L.H;
+    CUDA_TRY(cudaMemcpyAsync(dx, x_host, bytes, cudaMemcpyHostToDevice, st));
+    int rc = moe_forward(h, dx, T, dout, stream);
+    if (rc != MOE_OK) return rc;
+    CUDA_TRY(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return MOE_OK;
+}
+
+int moe_route(moe_handle* h, const uint16_t* x, int32_t T, int32_t* idx, float* gates, float* shared_gate,
+              int32_t* offsets, int32_t* perm, void* stream) {
+    int rc = check_call(h, x, T, nullptr, false);
+    if (rc != MOE_OK || T == 0) return rc;
+    DeviceGuard guard(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    const bool decode = use_decode(h, T);
+    Ctx c = make_ctx(h, T, x, nullptr, decode);
+    // the decode path's split-K router, then the prefill bucketing (so offsets/perm exist for any T)
+    CUDA_TRY(launch_router_simt(c, st));
+    CUDA_TRY(launch_topk(c, true, st));
+    CUDA_TRY(launch_bucket_scan(c, st));
+    CUDA_TRY(launch_scatter(c, st));
+    const Layout& L = h->L;
+    if (idx) CUDA_TRY(cudaMemcpyAsync(idx, c.idx, sizeof(int) * (size_t)T * L.k, cudaMemcpyDeviceToDevice, st));
+    if (gates) CUDA_TRY(cudaMemcpyAsync(gates, c.gates, sizeof(float) * (size_t)T * L.k, cudaMemcpyDeviceToDevice, st));
+    if (shared_gate) CUDA_TRY(cudaMemcpyAsync(shared_gate, c.sg, sizeof(float) * (size_t)T, cudaMemcpyDeviceToDevice, st));
+    if (offsets) CUDA_TRY(cudaMemcpyAsync(offsets, c.offsets, sizeof(int) * (size_t)(L.E + 1), cudaMemcpyDeviceToDevice, st));
+    if (perm) CUDA_TRY(cudaMemcpyAsync(perm, c.perm, sizeof(int) * (size_t)T * L.k, cudaMemcpyDeviceToDevice, st));
+    return MOE_OK;
+}
+
+int moe_status(moe_handle* h) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+    DeviceGuard guard(h->device);
+    CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+    uint32_t s = 0;
+    CUDA_TRY(cudaMemcpy(&s, h->base.status, sizeof s, cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemset(h->base.status, 0, sizeof s));
+    if (s & MOE_STATUS_TIMEOUT) return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
+    if (s & MOE_STATUS_BOUNDS) return fail(MOE_ERR_DEVICE_BOUNDS, "a device-side index check failed");
+    if (s & MOE_STATUS_RANGE) return fail(MOE_ERR_RANGE, "a value exceeded the fp16 operand range");
+    return MOE_OK;
+}
+
+int moe_debug_copy(moe_handle* h, int which, void* dst, size_t bytes, void* stream) {
+    if (!h || !dst) return fail(MOE_ERR_INVALID_ARG, "handle or dst is NULL");
+    const Layout& L = h->L;
+    const void* src = nullptr;
+    size_t cap = 0;
+    switch (which) {
+        case 0: src = h->base.act; cap = sizeof(__half) * (size_t)L.rows_cap * L.I; break;
+        case 1: src = h->base.xp; cap = sizeof(__half) * (size_t)L.rows_cap * L.H; break;
+        case 2: src = h->base.part; cap = sizeof(float) * (size_t)L.Tm * L.E; break;
+        case 3: src = h->base.acc; cap = sizeof(float) * (size_t)L.Tm * L.H; break;
+        default: return fail(MOE_ERR_INVALID_ARG, "unknown buffer %d", which);
+    }
+    if (bytes > cap) return fail(MOE_ERR_INVALID_ARG, "%zu bytes exceed the buffer (%zu)", bytes, cap);
+    DeviceGuard guard(h->device);
+    CUDA_TRY(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+int moe_profile_enable(moe_handle* h, int enable) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+    DeviceGuard guard(h->device);
+    if (enable && !h->prof_ev) {
+        h->prof_ev = new cudaEvent_t[kProfCalls * kProfEvents]();
+        for (int i = 0; i < kProfCalls * kProfEvents; ++i) CUDA_TRY(cudaEventCreate(&h->prof_ev[i]));
+    }
+    h->prof = enable != 0;
+    h->prof_calls = 0;
+    return MOE_OK;
+}
+
+int moe_profile_read(moe_handle* h, float* ms, int32_t* launches) {
+    if (!h || !ms || !launches) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+    for (int i = 0; i < MOE_PROF_SLOTS; ++i) {
+        ms[i] = 0.f;
+        launches[i] = 0;
+    }
+    if (!h->prof_ev) return MOE_OK;
+    DeviceGuard guard(h->device);
+    for (int cidx = 0; cidx < h->prof_calls; ++cidx) {
+        for (int n = 1; n < h->prof_nev[cidx]; ++n) {
+            cudaEvent_t a = h->prof_ev[cidx * kProfEvents + n - 1], b = h->prof_ev[cidx * kProfEvents + n];
+            CUDA_TRY(cudaEventSynchronize(b));
+            float t = 0.f;
+            CUDA_TRY(cudaEventElapsedTime(&t, a, b));
+            const int slot = h->prof_slot[cidx][n];
+            if (slot >= 0 && slot < MOE_PROF_SLOTS) {
+                ms[slot] += t;
+                launches[slot] += 1;
+            }
+        }
+    }
+    h->prof_calls = 0;
+    return MOE_OK;
+}
+
+void moe_destroy(moe_handle* h) {
+    if (!h) return;
+    {
+        DeviceGuard guard(h->device);
+        cudaDeviceSynchronize();
+        if (h->prof_ev) {
+            for (int i = 0; i < kProfCalls * kProfEvents; ++i) cudaEventDestroy(h->prof_ev[i]);
+            delete[] h->prof_ev;
+        }
+        if (h->wbuf) cudaFree(h->wbuf);
+        if (h->ws) cudaFree(h->ws);
+    }
+    delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,94 @@
+// kernels.h -- internal interface between the C-ABI host code (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Tile geometry of the prefill grouped GEMMs (tokens per tile = UMMA N).
+constexpr int kBN = 128;          // token columns per tile
+constexpr int kStages = 6;        // pipeline depth (smem stages == TMEM A-operand stages)
+constexpr int kTokPerBucketBlk = 64;  // tokens per routing/bucketing CTA
+constexpr int kRouterTT = 32;     // tokens per CTA in the SIMT router (prefill sizes)
+constexpr int kRouterTTSmall = 8; // tokens per CTA in the SIMT router (decode sizes)
+constexpr int kRouterKSlice = 32; // input columns per CTA in the split-K SIMT router
+
+struct RepackArgs {
+    const uint32_t* q[2];
+    const uint16_t* s[2];
+    const uint16_t* b[2];
+    const uint32_t* qs[2];
+    const uint16_t* ss[2];
+    const uint16_t* bs[2];
+    int E;             // routed experts (group E = shared)
+    int rows_per_mat;  // rows of one source matrix (I for gate/up, H for down)
+    int cols;          // input columns (H for gate/up, I for down)
+    int gateup;        // 1: interleave gate/up rows; 0: plain rows
+    uint8_t* dst;
+    uint32_t* inexact;
+};
+
+// Everything a forward-path kernel needs (passed by value).
+struct Ctx {
+    int T, H, I, E, k, G, has_shared;
+    int nblk;          // routing/bucketing CTAs for T tokens
+    int ks;            // K slices of the router partial logits
+    int max_tiles;     // capacity of each tile list
+    int rows_cap;      // row capacity of xp / act
+    uint32_t flags;
+    // weights, kernel layout
+    const uint8_t* w_gu;
+    const uint8_t* w_dn;
+    const float* wrt;
+    const float* rbias;
+    const float* sgw;
+    // call inputs / outputs
+    const uint16_t* x;
+    uint16_t* out;
+    // workspace
+    float* part;
+    int* idx;
+    float* gates;
+    float* sg;
+    int* hist;
+    int* counts;
+    int* offsets;
+    int4* tiles1;
+    int4* tiles2;
+    int* ntiles;
+    int* perm;
+    int* row_token;
+    float* row_gate;
+    __half* xp;
+    __half* act;
+    float* acc;
+    float* dact;
+    float* dscale;
+    uint32_t* status;
+    unsigned int* counters;
+};
+
+cudaError_t launch_repack(const RepackArgs& a, int groups, int m_tiles, int k_steps, cudaStream_t st);
+cudaError_t launch_router_prep(const float* router, const float* bias, const float* sgw, int H, int E,
+                               float* wrt, float* bias_out, float* sgw_out, cudaStream_t st);
+
+// routing + bucketing
+cudaError_t launch_router_simt(const Ctx& c, cudaStream_t st);
+cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
+cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st);
+cudaError_t launch_scatter(const Ctx& c, cudaStream_t st);
+
+// prefill grouped GEMMs
+cudaError_t launch_gemm_gateup(const Ctx& c, const CUtensorMap& tm_xp, int num_sms, cudaStream_t st);
+cudaError_t launch_gemm_down(const Ctx& c, const CUtensorMap& tm_act, int num_sms, cudaStream_t st);
+cudaError_t launch_finalize(const Ctx& c, cudaStream_t st);
+int gemm_smem_bytes(bool gateup);
+
+// decode sparse GEMV
+cudaError_t launch_gemv_gateup(const Ctx& c, cudaStream_t st);
+cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st);
+
+}  // namespace moe

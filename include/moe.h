@@ -1,0 +1,186 @@
+/*
+ * moe.h -- C ABI of libmoe: one 4-bit-weight mixture-of-experts layer on an NVIDIA B200 (sm_100a).
+ *
+ * What one forward call computes (for every token t of x[T, H]):
+ *   logits[e] = x_t . router[e] (+ router_bias[e])                        e = 0..E-1, fp32
+ *   S_t       = the top_k experts by logit, descending (equal logits: lower index first)
+ *   g_j       = softmax over all E logits, restricted to S_t and renormalised (sums to 1)
+ *   s_t       = sigmoid(x_t . shared_gate)                   (only when has_shared != 0)
+ *   FFN_e(x)  = W_down,e ( silu(W_gate,e x) * (W_up,e x) ),   silu(z) = z / (1 + exp(-z))
+ *   out_t     = sum_j g_j FFN_{S_t[j]}(x_t) + s_t FFN_shared(x_t),   rounded to bf16
+ * Each weight is  W[r][c] = q[r][c] * s[r][c/64] + b[r][c/64]  with a 4-bit code q and a per-
+ * (row, 64-column group) bf16 scale s and bias b ("asymmetric int4, group 64").
+ *
+ * Where this comes from.  "Perplexity Open-Sources Lily, a Qwen-Specific Mac Engine That Beats
+ * MLX-LM in Its Test", section "A runtime shaped around one model": each token is routed to eight
+ * of 256 experts plus a shared expert, and expert loads are uneven.  Same page, section "The
+ * optimizations follow the workload": during prefill the 4-bit weights are rebuilt inside the
+ * grouped matrix multiplication instead of being expanded into a full weight array, and expert
+ * routing stays on the GPU with no CPU synchronisation.  "A Rust + Metal Inference Engine for
+ * Qwen3.6-35B-A3B on Apple Silicon" (body) and the "perplexity-lily-engine" note (body, limits
+ * paragraph): decode is bound by weight bytes (the sparse GEMVs run near the memory wall).  The
+ * gating formula, the sigmoid shared gate, SwiGLU and the int4/g64/bf16 format are this
+ * library's layer definition; the pages do not spell them out.
+ *
+ * Conventions for every entry point below.
+ *  - All tensor pointers are DEVICE pointers owned by the caller (except moe_forward_host, which
+ *    takes host pointers).  The library never frees or retains caller memory beyond the call,
+ *    except that moe_create copies (repacks) the weights into memory the handle owns, so the
+ *    caller may free its weight buffers as soon as moe_create has returned and its stream has
+ *    been synchronised.
+ *  - "stream" is a cudaStream_t passed as void* (NULL = the legacy default stream).  Calls are
+ *    stream-ordered and asynchronous: they return after enqueueing work, with no host
+ *    synchronisation, no device-to-host copy and no allocation (moe_create and moe_forward_host
+ *    excepted).  Outputs are overwritten, never accumulated into.
+ *  - Return value: MOE_OK or one of the MOE_ERR_* codes.  No exception crosses the ABI.  An error
+ *    found before launch returns its code and launches nothing; a text message is then available
+ *    from moe_last_error() on the calling thread.  Errors found on the device (a timed-out wait,
+ *    an out-of-range index, a value outside the fp16 operand range) are recorded in a status word
+ *    and reported by the next moe_status() call.
+ *  - One stream at a time per handle: calls on one handle must not overlap on the device (they
+ *    share the handle's workspace).  Different handles are independent.
+ *  - Layouts are row-major and densely packed.  bf16 and fp16 values are passed as uint16 bit
+ *    patterns.  Pointers must be 16-byte aligned.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes ----------------------------------------------------------------------------- */
+#define MOE_OK                      0
+#define MOE_ERR_INVALID_ARG         1  /* null/misaligned pointer, unsupported shape, bad flag */
+#define MOE_ERR_UNSUPPORTED_DEVICE  2  /* device is not sm_100 (B200 class) */
+#define MOE_ERR_TOO_LARGE           3  /* T > max_tokens */
+#define MOE_ERR_CUDA                4  /* a CUDA runtime call failed (message in moe_last_error) */
+#define MOE_ERR_DEVICE_TIMEOUT      5  /* a bounded device-side wait ran out (kernel returned early) */
+#define MOE_ERR_DEVICE_BOUNDS       6  /* a device-side index check failed (access skipped) */
+#define MOE_ERR_RANGE               7  /* a value did not fit the fp16 tensor-core operand range */
+
+/* ---- configuration flags ---------------------------------------------------------------------- */
+#define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
+#define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its first load,
+                                          so the consumers' bounded waits run out and the call
+                                          reports MOE_ERR_DEVICE_TIMEOUT; nothing traps or hangs */
+
+typedef struct moe_handle moe_handle;
+
+/* Shapes of one layer.  Supported: hidden % 128 == 0, inter % 64 == 0, group == 64,
+ * 1 <= top_k <= num_experts <= 256, top_k <= 32, 1 <= max_tokens <= 65536. */
+typedef struct {
+    int32_t hidden;            /* H */
+    int32_t inter;             /* I: intermediate size of every expert, shared one included */
+    int32_t num_experts;       /* E: routed experts */
+    int32_t top_k;             /* k */
+    int32_t group;             /* quantisation group along the input dimension (must be 64) */
+    int32_t has_shared;        /* 1: one always-on shared expert with a sigmoid gate */
+    int32_t max_tokens;        /* largest T that moe_forward / moe_route accept */
+    int32_t decode_max_tokens; /* T <= this runs the sparse-GEMV decode path; larger T runs the
+                                  bucketed grouped-GEMM prefill path.  0 = always prefill path. */
+    uint32_t flags;            /* MOE_FLAG_* */
+} moe_config;
+
+/* Weights of one layer in the public ("natural") layout, all DEVICE pointers.
+ *  q_gate, q_up : uint32 [E, I, H/8]   packed codes; nibble j (bits 4j..4j+3) of word w is
+ *  q_down       : uint32 [E, H, I/8]   element 8w+j of the row (low nibble first)
+ *  s_*, b_*     : bf16   [E, rows, cols/64]  scale and bias of each 64-column group
+ *  qs_*, ss_*, bs_* : the shared expert, same layout without the leading E (NULL if no shared)
+ *  router       : fp32 [E, H];  router_bias: fp32 [E] or NULL;  shared_gate: fp32 [H] or NULL */
+typedef struct {
+    const uint32_t *q_gate, *q_up, *q_down;
+    const uint16_t *s_gate, *b_gate, *s_up, *b_up, *s_down, *b_down;
+    const uint32_t *qs_gate, *qs_up, *qs_down;
+    const uint16_t *ss_gate, *bs_gate, *ss_up, *bs_up, *ss_down, *bs_down;
+    const float *router;
+    const float *router_bias;
+    const float *shared_gate;
+} moe_weights;
+
+/* Create a layer on `device`: validate cfg, check the device is sm_100, allocate the handle's
+ * workspace (sized for cfg->max_tokens) and repack the weights into the handle's own kernel
+ * layout with kernels enqueued on `stream`.  moe_create synchronises `stream` before returning,
+ * so the caller may free its weight buffers as soon as it returns.  On success *out receives the
+ * handle.  Allocates device memory (the only entry point that does).  Scales/biases that are not
+ * exactly representable in fp16 are rounded to nearest (the layer still works; the tensor-core
+ * path computes in fp16).  Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+MOE_API int moe_create(const moe_config *cfg, const moe_weights *w, int device, void *stream,
+               moe_handle **out);
+
+/* out[T, H] (bf16) = the layer applied to x[T, H] (bf16), both device pointers.  T == 0 is a
+ * no-op returning MOE_OK.  Errors: INVALID_ARG (null/misaligned pointer, T < 0), TOO_LARGE
+ * (T > max_tokens), CUDA (launch failure).  Device-side errors surface via moe_status(). */
+MOE_API int moe_forward(moe_handle *h, const uint16_t *x, int32_t T, uint16_t *out, void *stream);
+
+/* The same with HOST buffers: copies x to the device, runs moe_forward, copies out back and
+ * synchronises `stream` before returning (so the host buffer is ready).  Pinned host memory is
+ * fastest; pageable memory works.  Uses handle-owned device staging buffers (no allocation). */
+MOE_API int moe_forward_host(moe_handle *h, const uint16_t *x_host, int32_t T, uint16_t *out_host,
+                     void *stream);
+
+/* Routing and bucketing only (the first steps of the prefill path), with their results copied
+ * to caller device buffers (any output pointer may be NULL to skip it):
+ *   idx[T, k] int32      experts per token, descending logit
+ *   gates[T, k] fp32     renormalised softmax gates, same order
+ *   shared_gate[T] fp32  sigmoid shared-expert gate (zeros when has_shared == 0)
+ *   offsets[E+1] int32   bucket starts: offsets[e] = number of (token, slot) entries routed to
+ *                        experts < e; offsets[E] = T*k
+ *   perm[T*k] int32      perm[p] = t*k + j for the entry at bucket position p; buckets are in
+ *                        expert order and each bucket lists its tokens in ascending order.
+ * Errors as for moe_forward. */
+MOE_API int moe_route(moe_handle *h, const uint16_t *x, int32_t T, int32_t *idx, float *gates,
+              float *shared_gate, int32_t *offsets, int32_t *perm, void *stream);
+
+/* Synchronise the stream of the handle's last call, read and clear the device status word.
+ * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS, MOE_ERR_RANGE (the most severe
+ * recorded, in that order of precedence reversed: timeout > bounds > range) or MOE_ERR_CUDA. */
+MOE_API int moe_status(moe_handle *h);
+
+/* Debug: copy `bytes` of an internal workspace buffer to a caller device buffer (stream-ordered).
+ * which: 0 = expert activations act[rows, I] (fp16, bucket order, prefill path),
+ *        1 = gathered input rows xp[rows, H] (fp16, bucket order),
+ *        2 = router logits [T, E] (fp32, tensor-core router only),
+ *        3 = fp32 combine accumulator [T, H].
+ * Errors: INVALID_ARG when `which` is unknown or `bytes` exceeds the buffer. */
+MOE_API int moe_debug_copy(moe_handle *h, int which, void *dst, size_t bytes, void *stream);
+
+/* Per-kernel timing.  While enabled, moe_forward records a CUDA event on the call's stream before
+ * its first kernel and after each kernel it launches (events are created by moe_profile_enable;
+ * up to 1024 calls are recorded, later calls run unrecorded).  Do not enable it while capturing a
+ * CUDA graph.  moe_profile_read synchronises those events, writes per kernel slot the summed
+ * device time in milliseconds (ms[MOE_PROF_SLOTS]) and the number of launches
+ * (launches[MOE_PROF_SLOTS]), and clears the record.  Slots: 0 router logits, 1 top-k and gates,
+ * 2 bucket scan, 3 scatter/gather, 4 gate/up grouped GEMM, 5 down grouped GEMM + combine,
+ * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine.
+ * Errors: INVALID_ARG, CUDA. */
+#define MOE_PROF_SLOTS 9
+MOE_API int moe_profile_enable(moe_handle *h, int enable);
+MOE_API int moe_profile_read(moe_handle *h, float *ms, int32_t *launches);
+
+/* Bytes of device memory a handle with this configuration owns (repacked weights + workspace). */
+MOE_API size_t moe_device_bytes(const moe_config *cfg);
+
+/* Message describing the last error returned on the calling thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+/* Free the handle and all device memory it owns.  Synchronises the device first.  NULL is a no-op. */
+MOE_API void moe_destroy(moe_handle *h);
+
+/* Library version as major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

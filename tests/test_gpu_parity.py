@@ -1,0 +1,211 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200).
+
+Expert indices, bucket offsets and the bucket permutation must match the oracle bit for bit (the
+activations are drawn so the top-(k+1) fp64 logits of every token are >= 1e-3 apart); gates to
+fp32 accuracy; layer outputs within the tolerance in tests/parity.py.  Sizes: the tiny layer and
+small ragged shapes span several tiles and a ragged tail; the full workloads (T = 1, 512, 4096)
+are compared on every token's routing and on all (T <= 512) or a seeded sample of 256 tokens'
+outputs, in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_grouped_expert_router_b200 import _lib as M
+from bit_grouped_expert_router_b200 import build as B
+from bit_grouped_expert_router_b200 import synth
+from helpers import gapped_x
+from parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    B.build()
+    M.lib()
+
+
+def _cuda(w):
+    return {k: (v.cuda() if v is not None else None) for k, v in w.items()}
+
+
+def _layer(w, shape, **kw):
+    return M.Layer.from_shape(_cuda(w), shape, **kw)
+
+
+def _route_check(layer, ol, x, shape):
+    r = layer.route(x.cuda())
+    torch.cuda.synchronize()
+    idx, g, sg, _ = ol.route(x)
+    assert (r["idx"].cpu().numpy() == idx).all(), "expert indices differ"
+    np.testing.assert_allclose(r["gates"].cpu().numpy(), g, rtol=1e-5, atol=2e-6)
+    if shape.has_shared:
+        np.testing.assert_allclose(r["shared_gate"].cpu().numpy(), sg, rtol=1e-5, atol=2e-6)
+    _, off, perm = oracle.bucket(idx, shape.E)
+    assert (r["offsets"].cpu().numpy() == off).all(), "bucket offsets differ"
+    assert (r["perm"].cpu().numpy() == perm).all(), "bucket permutation differs"
+    assert layer.status() == M.MOE_OK
+
+
+def _forward_check(layer, ol, x, tokens=None):
+    out = layer.forward(x.cuda())
+    torch.cuda.synchronize()
+    assert layer.status() == M.MOE_OK
+    ref = ol.forward(x, tokens=tokens)
+    got = out.cpu() if tokens is None else out.cpu()[torch.as_tensor(tokens, dtype=torch.long)]
+    return compare(got, ref)
+
+
+# ---------------------------------------------------------------------------------------------
+# tiny layer and small ragged shapes: both paths, every token
+TINY = synth.WORKLOADS["tiny"]
+RAGGED = synth.Shape("ragged", T=300, H=512, E=32, k=4, I=256, zipf_s=1.1, seed=21)
+NOSHARED = synth.Shape("noshared", T=77, H=256, E=16, k=2, I=128, has_shared=False, seed=22)
+KEQE = synth.Shape("k_eq_e", T=40, H=256, E=8, k=8, I=128, seed=23)
+SINGLE = synth.Shape("single", T=130, H=256, E=1, k=1, I=192, has_shared=False, seed=24)
+
+
+@pytest.mark.parametrize("shape", [TINY, RAGGED, NOSHARED, KEQE, SINGLE], ids=lambda s: s.name)
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+def test_small_shapes(shape, path):
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    dec = 0 if path == "prefill" else shape.T
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=dec)
+    _route_check(layer, ol, x, shape)
+    _forward_check(layer, ol, x)
+    # every prefix length exercises ragged tiles: 1, a tile boundary +/- 1 and the whole
+    for T in sorted({1, 2, min(shape.T, 17), min(shape.T, 128), min(shape.T, 129), shape.T}):
+        _forward_check(layer, ol, x[:T])
+    layer.close()
+
+
+def test_tiny_intermediate_activations_match():
+    """The gate/up GEMM alone: act rows in bucket order vs silu(Wg x) * (Wu x) from the oracle's
+    dequantised weights (fp64), within fp16 rounding."""
+    shape = TINY
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=0)
+    layer.forward(x.cuda())
+    rows = shape.T * shape.k + shape.T
+    act = torch.empty((rows, shape.I), dtype=torch.float16, device="cuda")
+    layer.debug_copy(0, act)
+    torch.cuda.synchronize()
+    idx, _, _, _ = ol.route(x)
+    _, _, perm = oracle.bucket(idx, shape.E)
+    X = x.float().double().numpy()
+    for p in range(rows):
+        if p < shape.T * shape.k:
+            t, e = perm[p] // shape.k, idx.ravel()[perm[p]]
+            sfx, ee = "", e
+        else:
+            t, sfx, ee = p - shape.T * shape.k, "s", None
+        def dq(n):
+            q, s, b = w["q" + sfx + "_" + n], w["s" + sfx + "_" + n], w["b" + sfx + "_" + n]
+            if ee is not None:
+                q, s, b = q[ee], s[ee], b[ee]
+            return oracle.dequant(q, s, b, shape.I, shape.H).astype(np.float64)
+        gz = dq("gate") @ X[t]
+        ref = gz / (1 + np.exp(-gz)) * (dq("up") @ X[t])
+        got = act[p].float().double().cpu().numpy()
+        np.testing.assert_allclose(got, ref, rtol=2e-3, atol=2e-3)
+    layer.close()
+
+
+# ---------------------------------------------------------------------------------------------
+# full-size workloads in the benchmark's launch configuration
+def _full(name, layer_idx=0, chunk=0, T=None):
+    shape = synth.WORKLOADS[name]
+    w = synth.make_layer(shape, layer_idx)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol, layer_idx, chunk, T)
+    return shape, w, ol, x
+
+
+def _sample(T, n, seed):
+    if T <= n:
+        return None
+    return sorted(np.random.default_rng(seed).choice(T, n, replace=False).tolist())
+
+
+@pytest.mark.parametrize("name,layer_idx,chunk", [("prefill512", 0, 0), ("prefill4k_zipf", 0, 0),
+                                                  ("prefill16k_zipf", 0, 0), ("prefill16k_zipf", 39, 3)])
+def test_full_prefill_workloads(name, layer_idx, chunk):
+    shape, w, ol, x = _full(name, layer_idx, chunk)
+    layer = _layer(w, shape, max_tokens=4096, decode_max_tokens=16)
+    _route_check(layer, ol, x, shape)
+    stats = _forward_check(layer, ol, x, tokens=_sample(shape.T, 256, 7 + layer_idx))
+    print(name, stats)
+    layer.close()
+
+
+@pytest.mark.parametrize("layer_idx", [0, 39])
+def test_full_decode_workload(layer_idx):
+    shape, w, ol, x = _full("decode", layer_idx, 0, T=16)
+    layer = _layer(w, shape, max_tokens=4096, decode_max_tokens=16)
+    _route_check(layer, ol, x[:1], shape)
+    print("decode T=1", _forward_check(layer, ol, x[:1]))
+    print("decode T=16", _forward_check(layer, ol, x))
+    # the same tokens through the prefill path agree too
+    layer2 = _layer(w, shape, max_tokens=4096, decode_max_tokens=0)
+    print("prefill T=16", _forward_check(layer2, ol, x))
+    layer.close()
+    layer2.close()
+
+
+def test_forced_experts_make_large_buckets():
+    shape = synth.Shape("forced", T=1024, H=2048, E=256, k=8, I=512, seed=31)
+    w = synth.make_layer(shape)
+    chosen = [3, 40, 77, 100, 150, 201, 222, 255]
+    bias = torch.zeros(shape.E)
+    bias[chosen] = 100.0
+    w["router_bias"] = bias
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    layer = _layer(w, shape, max_tokens=1024, decode_max_tokens=0)
+    _route_check(layer, ol, x, shape)
+    _forward_check(layer, ol, x, tokens=_sample(shape.T, 64, 3))
+    layer.close()
+
+
+# ---------------------------------------------------------------------------------------------
+# boundary behaviour through the C ABI
+def test_host_buffers_and_edge_calls():
+    shape = TINY
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=2)
+    dev = layer.forward(x.cuda()).cpu()
+    host = layer.forward_host(x.pin_memory())
+    assert torch.equal(dev.view(torch.int16), host.view(torch.int16))
+    # T = 0 is a no-op, T > max_tokens is refused before launch
+    assert M.lib().moe_forward(layer.handle, x.cuda().data_ptr(), 0, None, None) == M.MOE_OK
+    out = torch.empty((shape.T + 1, shape.H), dtype=torch.bfloat16, device="cuda")
+    xx = torch.zeros((shape.T + 1, shape.H), dtype=torch.bfloat16, device="cuda")
+    rc = M.lib().moe_forward(layer.handle, xx.data_ptr(), shape.T + 1, out.data_ptr(), None)
+    assert rc == M.MOE_ERR_TOO_LARGE
+    # misaligned pointer
+    rc = M.lib().moe_forward(layer.handle, xx.data_ptr() + 2, 1, out.data_ptr(), None)
+    assert rc == M.MOE_ERR_INVALID_ARG
+    assert layer.status() == M.MOE_OK
+    layer.close()
+
+
+def test_fp16_range_overflow_is_reported():
+    shape = synth.shape_with(TINY, T=4)
+    w = synth.make_layer(shape)
+    layer = _layer(w, shape, max_tokens=4, decode_max_tokens=0)
+    x = torch.zeros((4, shape.H), dtype=torch.bfloat16)
+    x[1, 5] = 1.0e6   # representable in bf16, not in fp16
+    layer.forward(x.cuda())
+    assert layer.status() == M.MOE_ERR_RANGE
+    assert layer.status() == M.MOE_OK   # cleared
+    layer.close()
