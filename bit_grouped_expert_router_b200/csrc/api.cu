@@ -61,8 +61,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Sizes derived from a configuration.
 struct Layout {
-    int H, I, E, k, G, Tm, Tdec, ks_dec, nblk_max, max_tiles, rows_cap;
-    size_t w_gu_bytes, w_dn_bytes, router_bytes, weights_bytes;
+    int H, I, E, k, G, Tm, Tdec, ks_dec, nblk_max, max_tiles, rows_cap, Epad;
+    size_t w_gu_bytes, w_dn_bytes, router_bytes, wsplit_bytes, weights_bytes;
     // workspace offsets
     size_t o_part, o_idx, o_gates, o_sg, o_hist, o_counts, o_offsets, o_tiles, o_ntiles, o_perm, o_rtok,
         o_rgate, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_counters, o_stage_x, o_stage_out, ws_bytes;
@@ -87,7 +87,10 @@ Layout make_layout(const moe_config& c) {
     L.w_gu_bytes = per_mat_gu * L.G;
     L.w_dn_bytes = per_mat_dn * L.G;
     L.router_bytes = sizeof(float) * ((size_t)L.H * L.E + L.E + L.H);
-    L.weights_bytes = align_up(L.w_gu_bytes, 256) + align_up(L.w_dn_bytes, 256) + align_up(L.router_bytes, 256);
+    L.Epad = (L.E + 127) / 128 * 128;
+    L.wsplit_bytes = sizeof(uint16_t) * (size_t)L.Epad * 2 * L.H;
+    L.weights_bytes = align_up(L.w_gu_bytes, 256) + align_up(L.w_dn_bytes, 256) + align_up(L.router_bytes, 256) +
+                      align_up(L.wsplit_bytes, 256);
 
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -154,15 +157,16 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 2-D fp16 row-major [rows, cols] tensor, box {64 columns, box_rows rows}, 128-byte swizzle.
-int encode_rows_map(CUtensorMap* m, void* base, int rows, int cols, int box_rows) {
+// 2-D 16-bit row-major [rows, cols] tensor, box {64 columns, box_rows rows}, 128-byte swizzle.
+int encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows,
+                    CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr,
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -188,7 +192,8 @@ struct moe_handle {
     uint8_t* wbuf = nullptr;
     uint8_t* ws = nullptr;
     Ctx base{};
-    CUtensorMap tm_xp{}, tm_act{};
+    CUtensorMap tm_xp{}, tm_act{}, tm_wsplit{};
+    uint16_t* wsplit = nullptr;
     cudaStream_t last_stream = nullptr;
     bool inexact_scales = false;
 };
@@ -239,8 +244,15 @@ struct Prof {
     }
 };
 
-int enqueue_routing(Prof& pf, const Ctx& c, bool decode, cudaStream_t st) {
-    CUDA_TRY(launch_router_simt(c, st));
+int enqueue_routing(moe_handle* h, Prof& pf, const Ctx& c, bool decode, cudaStream_t st) {
+    if (decode || (h->cfg.flags & MOE_FLAG_ROUTER_SIMT)) {
+        CUDA_TRY(launch_router_simt(c, st));
+    } else {
+        CUtensorMap tm_x;
+        const int rc = encode_rows_map(&tm_x, c.x, c.T, c.H, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        if (rc != MOE_OK) return rc;
+        CUDA_TRY(launch_router_tc(c, h->tm_wsplit, tm_x, h->L.Epad / 128, st));
+    }
     pf.mark(0);
     CUDA_TRY(launch_topk(c, !decode, st));
     pf.mark(1);
@@ -321,6 +333,8 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     float* wrt = reinterpret_cast<float*>(w_dn + align_up(L.w_dn_bytes, 256));
     float* rbias = wrt + (size_t)L.H * L.E;
     float* sgw = rbias + L.E;
+    uint16_t* wsplit = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(wrt) + align_up(L.router_bytes, 256));
+    h->wsplit = wsplit;
     uint32_t* status = reinterpret_cast<uint32_t*>(h->ws + L.o_status);
 
     RepackArgs a{};
@@ -352,6 +366,8 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     e = launch_router_prep(w->router, w->router_bias, cfg->has_shared ? w->shared_gate : nullptr, L.H, L.E, wrt, rbias,
                            sgw, st);
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router prep: %s", cudaGetErrorString(e)));
+    e = launch_router_split(w->router, L.H, L.E, L.Epad, wsplit, st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router split: %s", cudaGetErrorString(e)));
     uint32_t flags_host[2] = {0, 0};
     e = cudaMemcpyAsync(flags_host, status, sizeof flags_host, cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -391,6 +407,8 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
 
     rc = encode_rows_map(&h->tm_xp, c.xp, L.rows_cap, L.H, kBN);
     if (rc == MOE_OK) rc = encode_rows_map(&h->tm_act, c.act, L.rows_cap, L.I, kBN);
+    if (rc == MOE_OK)
+        rc = encode_rows_map(&h->tm_wsplit, wsplit, L.Epad, 2 * L.H, 128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc != MOE_OK) return cleanup(rc);
     h->last_stream = st;
     *out = h;
@@ -406,7 +424,7 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     const bool decode = use_decode(h, T);
     const Ctx c = make_ctx(h, T, x, out, decode);
     Prof pf(h, st);
-    rc = enqueue_routing(pf, c, decode, st);
+    rc = enqueue_routing(h, pf, c, decode, st);
     if (rc != MOE_OK) return rc;
     if (decode) {
         CUDA_TRY(launch_gemv_gateup(c, st));
@@ -452,11 +470,17 @@ int moe_route(moe_handle* h, const uint16_t* x, int32_t T, int32_t* idx, float* 
     h->last_stream = st;
     const bool decode = use_decode(h, T);
     Ctx c = make_ctx(h, T, x, nullptr, decode);
-    // the decode path's split-K router, then the prefill bucketing (so offsets/perm exist for any T)
-    CUDA_TRY(launch_router_simt(c, st));
-    CUDA_TRY(launch_topk(c, true, st));
-    CUDA_TRY(launch_bucket_scan(c, st));
-    CUDA_TRY(launch_scatter(c, st));
+    // the router the forward call would use for this T, then the prefill bucketing (so offsets
+    // and perm exist for any T)
+    Prof pf(h, st);
+    pf.call = -1;
+    rc = enqueue_routing(h, pf, c, decode, st);
+    if (rc != MOE_OK) return rc;
+    if (decode) {
+        CUDA_TRY(launch_topk(c, true, st));
+        CUDA_TRY(launch_bucket_scan(c, st));
+        CUDA_TRY(launch_scatter(c, st));
+    }
     const Layout& L = h->L;
     if (idx) CUDA_TRY(cudaMemcpyAsync(idx, c.idx, sizeof(int) * (size_t)T * L.k, cudaMemcpyDeviceToDevice, st));
     if (gates) CUDA_TRY(cudaMemcpyAsync(gates, c.gates, sizeof(float) * (size_t)T * L.k, cudaMemcpyDeviceToDevice, st));

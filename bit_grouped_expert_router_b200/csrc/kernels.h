@@ -77,6 +77,10 @@ cudaError_t launch_router_prep(const float* router, const float* bias, const flo
 
 // routing + bucketing
 cudaError_t launch_router_simt(const Ctx& c, cudaStream_t st);
+cudaError_t launch_router_split(const float* router, int H, int E, int Epad, uint16_t* wsplit, cudaStream_t st);
+cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmA, const CUtensorMap& tmB, int mtiles,
+                             cudaStream_t st);
+int router_tc_smem_bytes();
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
 cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st);
