@@ -79,8 +79,9 @@ def lib() -> ctypes.CDLL:
         L.moe_version.restype = ctypes.c_int
         L.moe_profile_enable.argtypes = [P, ctypes.c_int]
         L.moe_profile_read.argtypes = [P, P, P]
+        L.moe_route_static.argtypes = [P, I32, I32, P, P, I32, I32, P, P, P]
         for n in ("moe_create", "moe_forward", "moe_forward_host", "moe_route", "moe_status",
-                  "moe_debug_copy", "moe_profile_enable", "moe_profile_read"):
+                  "moe_debug_copy", "moe_profile_enable", "moe_profile_read", "moe_route_static"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib

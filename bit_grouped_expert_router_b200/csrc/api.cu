@@ -175,6 +175,8 @@ int encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int bo
 
 }  // namespace
 
+void moe::set_last_error(const char* msg) { g_last_error = msg; }
+
 constexpr int kProfCalls = 1024;
 constexpr int kProfEvents = 8;  // at most 7 kernels per call + the leading event
 

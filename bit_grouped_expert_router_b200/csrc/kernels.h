@@ -91,6 +91,9 @@ cudaError_t launch_gemm_down(const Ctx& c, const CUtensorMap& tm_act, int num_sm
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st);
 int gemm_smem_bytes(bool gateup);
 
+// host-side error text for moe_last_error() (defined in api.cu)
+void set_last_error(const char* msg);
+
 // decode sparse GEMV
 cudaError_t launch_gemv_gateup(const Ctx& c, cudaStream_t st);
 cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st);

@@ -176,6 +176,27 @@ MOE_API const char *moe_last_error(void);
 /* Free the handle and all device memory it owns.  Synchronises the device first.  NULL is a no-op. */
 MOE_API void moe_destroy(moe_handle *h);
 
+/* Routing for callers that cannot allocate device memory.  No counterpart on the pages: this is a
+ * library convenience.  Some callers may not call cudaMalloc at all -- a thread recording a CUDA
+ * graph (allocation is not a stream operation), a latency-critical serving loop kept out of the
+ * allocator, a plug-in inside a framework that owns every device allocation -- and so cannot
+ * create a moe_handle.  This entry point computes, for x[T, H] (bf16, device), the router's top-k
+ * experts idx[T, k] (int32, device) and their renormalised gates gates[T, k] (fp32, device) from
+ * the caller's router[E, H] (fp32, device, public layout) and optional router_bias[E] (fp32 or
+ * NULL), exactly as moe_route does, on the current device and `stream`.  It allocates nothing:
+ * its only scratch (split-K partial logits, T * (H/32) * E floats) lives in a fixed array of
+ * MOE_ROUTE_STATIC_SCRATCH_FLOATS floats (1 MiB) compiled into the library, which every GPU that
+ * loads the library holds until the process exits.  Larger requests return MOE_ERR_TOO_LARGE.
+ * The array is shared by all calls and keeps the last call's contents (each call overwrites what
+ * it reads, so nothing needs clearing); calls that overlap on the GPU race on it -- serialise
+ * them.  The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture begins.
+ * Errors: INVALID_ARG (H % 32 != 0, k or E out of range, NULL pointer), TOO_LARGE, CUDA. */
+#define MOE_ROUTE_STATIC_SCRATCH_FLOATS 262144
+MOE_API int moe_route_static(const uint16_t *x, int32_t T, int32_t H, const float *router,
+                             const float *router_bias, int32_t E, int32_t k, int32_t *idx,
+                             float *gates, void *stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 MOE_API int moe_version(void);
 
