@@ -261,7 +261,7 @@ def run_prefill(args, dist, peaks, peak_src):
         gg = {"achieved_tflops": round(a, 1), "frac_of_peak": round(a / peak_tf, 4),
               "us_per_chunk": round(t * 1e6, 1)}
     res = dict(value=value, ms=ms, clocks=clk, roofline=roof, kernels=prof, grouped_gemm=gg,
-               launches=7 * chunks * n_layers * args.steps, shape=shape, n_layers=n_layers,
+               launches=8 * chunks * n_layers * args.steps, shape=shape, n_layers=n_layers,
                tokens_per_step=tokens_per_step)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
@@ -316,7 +316,13 @@ def run_decode(args, dist, peaks, peak_src):
     nexp = shape.k + 1
     hbm = peaks["hbm_gbs"]
     roof = None
-    if "gemv_gateup" in prof and "gemv_down" in prof:
+    if "decode_fused" in prof:
+        b = nexp * expert_bytes + shape.E * shape.H * 4 + shape.H * 4 + 2 * shape.H * 2
+        a = b / (prof["decode_fused"]["avg_us"] * 1e-6) / 1e9
+        roof = {"bound": "hbm", "kernel": "single-kernel batch-1 decode (eager, profiled)",
+                "achieved": round(a, 1), "peak": hbm, "unit": "GB/s", "frac": round(a / hbm, 4),
+                "traffic": None, "bytes_per_token": b, "peak_source": f"{peak_src} hbm_gbs"}
+    elif "gemv_gateup" in prof and "gemv_down" in prof:
         b_gu = nexp * (shape.I // 64) * (shape.H // 64) * 4608 + shape.H * 2
         b_dn = nexp * (shape.H // 128) * (shape.I // 64) * 4608 + shape.H * 2
         t = (prof["gemv_gateup"]["avg_us"] + prof["gemv_down"]["avg_us"]) * 1e-6
@@ -334,7 +340,7 @@ def run_decode(args, dist, peaks, peak_src):
             "value": round(us_layer, 3), "unit": "us/token/layer", "higher_is_better": False,
             "whole_layer_hbm_frac": round(layer_bytes / (us_layer * 1e-6) / 1e9 / hbm, 4),
             "whole_layer_bytes": layer_bytes, "roofline": roof, "kernels": prof,
-            "gpu_launches_per_step": 4 * n_layers}
+            "gpu_launches_per_step": (1 if "decode_fused" in prof else 4) * n_layers}
 
 
 # ------------------------------------------------------------------------------------ CPU oracle

@@ -25,6 +25,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_DEVICE_BOUNDS = 6
 MOE_ERR_RANGE = 7
 MOE_FLAG_ROUTER_SIMT = 0x1
+MOE_FLAG_DECODE_UNFUSED = 0x2
 MOE_FLAG_TEST_STALL = 0x100
 
 _ERR_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DEVICE", 3: "TOO_LARGE", 4: "CUDA",
@@ -186,7 +187,7 @@ class Layer:
         return dst
 
     PROF_SLOTS = ["router", "topk", "bucket_scan", "scatter", "gemm_gateup", "gemm_down", "finalize",
-                  "gemv_gateup", "gemv_down"]
+                  "gemv_gateup", "gemv_down", "decode_fused", "gather_rows"]
 
     def profile(self, enable: bool = True):
         check(lib().moe_profile_enable(self.handle, 1 if enable else 0))

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["api.cu", "repack.cu", "route.cu", "router_tc.cu", "gemm.cu", "decode.cu", "route_static.cu"]
+SOURCES = ["api.cu", "repack.cu", "route.cu", "router_tc.cu", "gemm.cu", "decode.cu", "decode_fused.cu", "route_static.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE]
 

@@ -2,9 +2,10 @@
 // sequence of one forward call.  Host code only; every step of the layer runs in the kernels.
 //
 // Prefill path (T > decode_max_tokens), all stream-ordered, no host synchronisation:
-//   router logits -> top-k/gates/histogram -> bucket scan + tile list -> scatter (bucketed fp16
-//   rows, zeroed accumulator) -> tcgen05 gate/up GEMM + SwiGLU -> tcgen05 down GEMM + combine
-//   -> bf16 finalize.
+//   tensor-core router logits -> top-k/gates/histogram (+ fp16 activation rows, zeroed
+//   accumulator) -> bucket scan + tile list -> scatter (bucket row -> token, gate) -> gather of
+//   the token rows into bucket order -> tcgen05 gate/up GEMM + SwiGLU -> tcgen05 down GEMM +
+//   combine -> bf16 finalize.
 // Decode path (T <= decode_max_tokens): split-K router -> top-k/gates -> sparse GEMV gate/up +
 //   SwiGLU -> sparse GEMV down + gated combine (bf16 out).
 #include <cudaTypedefs.h>
@@ -63,10 +64,15 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
     int H, I, E, k, G, Tm, Tdec, ks_dec, nblk_max, max_tiles, rows_cap, Epad;
     size_t w_gu_bytes, w_dn_bytes, router_bytes, wsplit_bytes, weights_bytes;
+    size_t o_wrt, o_rbias, o_sgw, o_router32;   // offsets inside the router region
     // workspace offsets
     size_t o_part, o_idx, o_gates, o_sg, o_hist, o_counts, o_offsets, o_tiles, o_ntiles, o_perm, o_rtok,
-        o_rgate, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_counters, o_stage_x, o_stage_out, ws_bytes;
+        o_rgate, o_x16, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_counters, o_stage_x, o_stage_out, o_dfz_rpart,
+        o_dfz_gu, o_dfz_outacc, o_dfz_cnt, o_dfz_bar, ws_bytes;
 };
+
+struct Layout;
+int router_n_exp(const Layout& L);
 
 Layout make_layout(const moe_config& c) {
     Layout L{};
@@ -86,7 +92,13 @@ Layout make_layout(const moe_config& c) {
     const size_t per_mat_dn = (size_t)(L.H / 128) * (L.I / 64) * kBlockBytes;
     L.w_gu_bytes = per_mat_gu * L.G;
     L.w_dn_bytes = per_mat_dn * L.G;
-    L.router_bytes = sizeof(float) * ((size_t)L.H * L.E + L.E + L.H);
+    // router region: transposed fp32 [H][E], bias [E], shared-gate vector [H], public-layout fp32
+    // copy [E][H]; every sub-buffer starts on a 256-byte boundary (vector loads need 16 B)
+    L.o_wrt = 0;
+    L.o_rbias = align_up(L.o_wrt + sizeof(float) * (size_t)L.H * L.E, 256);
+    L.o_sgw = align_up(L.o_rbias + sizeof(float) * (size_t)L.E, 256);
+    L.o_router32 = align_up(L.o_sgw + sizeof(float) * (size_t)L.H, 256);
+    L.router_bytes = L.o_router32 + sizeof(float) * (size_t)L.H * L.E;
     L.Epad = (L.E + 127) / 128 * 128;
     L.wsplit_bytes = sizeof(uint16_t) * (size_t)L.Epad * 2 * L.H;
     L.weights_bytes = align_up(L.w_gu_bytes, 256) + align_up(L.w_dn_bytes, 256) + align_up(L.router_bytes, 256) +
@@ -98,7 +110,7 @@ Layout make_layout(const moe_config& c) {
         o = align_up(o + bytes, 256);
         return at;
     };
-    const size_t part_rows = std::max((size_t)L.Tm, (size_t)L.ks_dec * (size_t)L.Tdec);
+    const size_t part_rows = std::max((size_t)router_tc_splits() * L.Tm, (size_t)L.ks_dec * (size_t)L.Tdec);
     L.o_part = take(sizeof(float) * part_rows * L.E);
     L.o_idx = take(sizeof(int) * (size_t)L.Tm * L.k);
     L.o_gates = take(sizeof(float) * (size_t)L.Tm * L.k);
@@ -111,7 +123,8 @@ Layout make_layout(const moe_config& c) {
     L.o_perm = take(sizeof(int) * (size_t)L.Tm * L.k);
     L.o_rtok = take(sizeof(int) * (size_t)L.rows_cap);
     L.o_rgate = take(sizeof(float) * (size_t)L.rows_cap);
-    L.o_xp = take(sizeof(__half) * (size_t)L.rows_cap * L.H);
+    L.o_x16 = take(sizeof(__half) * (size_t)L.Tm * L.H);
+    L.o_xp = take(sizeof(__half) * (size_t)L.Tm * L.k * L.H);
     L.o_act = take(sizeof(__half) * (size_t)L.rows_cap * L.I);
     L.o_acc = take(sizeof(float) * (size_t)L.Tm * L.H);
     L.o_dact = take(sizeof(float) * (size_t)std::max(L.Tdec, 1) * (L.k + 1) * L.I);
@@ -120,9 +133,17 @@ Layout make_layout(const moe_config& c) {
     L.o_counters = take(sizeof(unsigned) * 64);
     L.o_stage_x = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
     L.o_stage_out = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
+    L.o_dfz_rpart = take(sizeof(float) * 4 * (size_t)L.E);
+    L.o_dfz_gu = take(sizeof(float) * (size_t)(L.k + 1) * 4 * 2 * L.I);
+    L.o_dfz_outacc = take(sizeof(float) * (size_t)L.H);
+    L.o_dfz_cnt = take(sizeof(unsigned) * (size_t)(L.H / 32));
+    L.o_dfz_bar = take(sizeof(unsigned) * 2);
     L.ws_bytes = o;
     return L;
 }
+
+// experts as the router GEMM's N: E rounded up to a multiple of 16
+int router_n_exp(const Layout& L) { return (L.E + 15) / 16 * 16; }
 
 int validate_config(const moe_config* c) {
     if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
@@ -135,7 +156,7 @@ int validate_config(const moe_config* c) {
     if (c->has_shared != 0 && c->has_shared != 1) return fail(MOE_ERR_INVALID_ARG, "has_shared must be 0 or 1");
     if (c->max_tokens < 1 || c->max_tokens > 65536) return fail(MOE_ERR_INVALID_ARG, "max_tokens must be in [1, 65536]");
     if (c->decode_max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "decode_max_tokens must be >= 0");
-    if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_TEST_STALL))
+    if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_DECODE_UNFUSED | MOE_FLAG_TEST_STALL))
         return fail(MOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
     return MOE_OK;
 }
@@ -178,7 +199,7 @@ int encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int bo
 void moe::set_last_error(const char* msg) { g_last_error = msg; }
 
 constexpr int kProfCalls = 1024;
-constexpr int kProfEvents = 8;  // at most 7 kernels per call + the leading event
+constexpr int kProfEvents = 9;  // at most 8 kernels per call + the leading event
 
 struct moe_handle {
     int device = 0;
@@ -194,7 +215,8 @@ struct moe_handle {
     uint8_t* wbuf = nullptr;
     uint8_t* ws = nullptr;
     Ctx base{};
-    CUtensorMap tm_xp{}, tm_act{}, tm_wsplit{};
+    TokenMaps maps_gu{}, maps_dn{};
+    CUtensorMap tm_wsplit{};
     uint16_t* wsplit = nullptr;
     cudaStream_t last_stream = nullptr;
     bool inexact_scales = false;
@@ -208,7 +230,7 @@ Ctx make_ctx(const moe_handle* h, int T, const uint16_t* x, uint16_t* out, bool 
     c.x = x;
     c.out = out;
     c.nblk = (T + kTokPerBucketBlk - 1) / kTokPerBucketBlk;
-    c.ks = decode ? h->L.ks_dec : 1;
+    c.ks = decode ? h->L.ks_dec : ((h->cfg.flags & MOE_FLAG_ROUTER_SIMT) ? 1 : router_tc_splits());
     return c;
 }
 
@@ -223,6 +245,11 @@ int check_call(moe_handle* h, const void* x, int32_t T, const void* out, bool ne
 }
 
 bool use_decode(const moe_handle* h, int T) { return T <= h->cfg.decode_max_tokens; }
+
+// The single-kernel decode handles T == 1 when its per-warp k-ranges fit (H <= 2048, I <= 2048).
+bool fused_decode_ok(const moe_handle* h) {
+    return !(h->cfg.flags & MOE_FLAG_DECODE_UNFUSED) && h->L.H / 64 <= 8 * 4 && h->L.I / 64 <= 8 * 4;
+}
 
 // Profiling: one event before the first kernel of a call and one after each kernel.
 struct Prof {
@@ -251,9 +278,9 @@ int enqueue_routing(moe_handle* h, Prof& pf, const Ctx& c, bool decode, cudaStre
         CUDA_TRY(launch_router_simt(c, st));
     } else {
         CUtensorMap tm_x;
-        const int rc = encode_rows_map(&tm_x, c.x, c.T, c.H, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        const int rc = encode_rows_map(&tm_x, c.x, c.T, c.H, 128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
         if (rc != MOE_OK) return rc;
-        CUDA_TRY(launch_router_tc(c, h->tm_wsplit, tm_x, h->L.Epad / 128, st));
+        CUDA_TRY(launch_router_tc(c, h->tm_wsplit, tm_x, router_n_exp(h->L), st));
     }
     pf.mark(0);
     CUDA_TRY(launch_topk(c, !decode, st));
@@ -332,10 +359,12 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
 
     uint8_t* w_gu = h->wbuf;
     uint8_t* w_dn = w_gu + align_up(L.w_gu_bytes, 256);
-    float* wrt = reinterpret_cast<float*>(w_dn + align_up(L.w_dn_bytes, 256));
-    float* rbias = wrt + (size_t)L.H * L.E;
-    float* sgw = rbias + L.E;
-    uint16_t* wsplit = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(wrt) + align_up(L.router_bytes, 256));
+    uint8_t* rregion = w_dn + align_up(L.w_dn_bytes, 256);
+    float* wrt = reinterpret_cast<float*>(rregion + L.o_wrt);
+    float* rbias = reinterpret_cast<float*>(rregion + L.o_rbias);
+    float* sgw = reinterpret_cast<float*>(rregion + L.o_sgw);
+    float* router32 = reinterpret_cast<float*>(rregion + L.o_router32);
+    uint16_t* wsplit = reinterpret_cast<uint16_t*>(rregion + align_up(L.router_bytes, 256));
     h->wsplit = wsplit;
     uint32_t* status = reinterpret_cast<uint32_t*>(h->ws + L.o_status);
 
@@ -368,6 +397,8 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     e = launch_router_prep(w->router, w->router_bias, cfg->has_shared ? w->shared_gate : nullptr, L.H, L.E, wrt, rbias,
                            sgw, st);
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router prep: %s", cudaGetErrorString(e)));
+    e = cudaMemcpyAsync(router32, w->router, sizeof(float) * (size_t)L.E * L.H, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router copy: %s", cudaGetErrorString(e)));
     e = launch_router_split(w->router, L.H, L.E, L.Epad, wsplit, st);
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router split: %s", cudaGetErrorString(e)));
     uint32_t flags_host[2] = {0, 0};
@@ -384,7 +415,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.max_tiles = L.max_tiles;
     c.rows_cap = L.rows_cap;
     c.flags = cfg->flags;
-    c.w_gu = w_gu; c.w_dn = w_dn; c.wrt = wrt; c.rbias = rbias; c.sgw = sgw;
+    c.w_gu = w_gu; c.w_dn = w_dn; c.wrt = wrt; c.rbias = rbias; c.sgw = sgw; c.router32 = router32;
     uint8_t* ws = h->ws;
     c.part = reinterpret_cast<float*>(ws + L.o_part);
     c.idx = reinterpret_cast<int*>(ws + L.o_idx);
@@ -399,6 +430,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.perm = reinterpret_cast<int*>(ws + L.o_perm);
     c.row_token = reinterpret_cast<int*>(ws + L.o_rtok);
     c.row_gate = reinterpret_cast<float*>(ws + L.o_rgate);
+    c.x16 = reinterpret_cast<__half*>(ws + L.o_x16);
     c.xp = reinterpret_cast<__half*>(ws + L.o_xp);
     c.act = reinterpret_cast<__half*>(ws + L.o_act);
     c.acc = reinterpret_cast<float*>(ws + L.o_acc);
@@ -406,11 +438,21 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.dscale = reinterpret_cast<float*>(ws + L.o_dscale);
     c.status = status;
     c.counters = reinterpret_cast<unsigned*>(ws + L.o_counters);
+    c.dfz.rpart = reinterpret_cast<float*>(ws + L.o_dfz_rpart);
+    c.dfz.gu = reinterpret_cast<float*>(ws + L.o_dfz_gu);
+    c.dfz.outacc = reinterpret_cast<float*>(ws + L.o_dfz_outacc);
+    c.dfz.cnt = reinterpret_cast<unsigned*>(ws + L.o_dfz_cnt);
+    c.dfz.bar = reinterpret_cast<unsigned*>(ws + L.o_dfz_bar);
 
-    rc = encode_rows_map(&h->tm_xp, c.xp, L.rows_cap, L.H, kBN);
-    if (rc == MOE_OK) rc = encode_rows_map(&h->tm_act, c.act, L.rows_cap, L.I, kBN);
+    for (int hs = 0; hs < 3 && rc == MOE_OK; ++hs) {
+        const int box = 64 << hs;
+        rc = encode_rows_map(&h->maps_gu.m[0][hs], c.xp, L.Tm * L.k, L.H, box);
+        if (rc == MOE_OK) rc = encode_rows_map(&h->maps_gu.m[1][hs], c.x16, L.Tm, L.H, box);
+        if (rc == MOE_OK) rc = encode_rows_map(&h->maps_dn.m[0][hs], c.act, L.rows_cap, L.I, box);
+        if (rc == MOE_OK) h->maps_dn.m[1][hs] = h->maps_dn.m[0][hs];
+    }
     if (rc == MOE_OK)
-        rc = encode_rows_map(&h->tm_wsplit, wsplit, L.Epad, 2 * L.H, 128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        rc = encode_rows_map(&h->tm_wsplit, wsplit, L.Epad, 2 * L.H, router_n_exp(L), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc != MOE_OK) return cleanup(rc);
     h->last_stream = st;
     *out = h;
@@ -426,6 +468,11 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     const bool decode = use_decode(h, T);
     const Ctx c = make_ctx(h, T, x, out, decode);
     Prof pf(h, st);
+    if (decode && T == 1 && fused_decode_ok(h)) {
+        CUDA_TRY(launch_decode_fused(c, h->num_sms, st));
+        pf.mark(9);
+        return MOE_OK;
+    }
     rc = enqueue_routing(h, pf, c, decode, st);
     if (rc != MOE_OK) return rc;
     if (decode) {
@@ -434,9 +481,11 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
         CUDA_TRY(launch_gemv_down(c, st));
         pf.mark(8);
     } else {
-        CUDA_TRY(launch_gemm_gateup(c, h->tm_xp, h->num_sms, st));
+        CUDA_TRY(launch_gather_rows(c, h->num_sms, st));
+        pf.mark(10);
+        CUDA_TRY(launch_gemm_gateup(c, h->maps_gu, h->num_sms, st));
         pf.mark(4);
-        CUDA_TRY(launch_gemm_down(c, h->tm_act, h->num_sms, st));
+        CUDA_TRY(launch_gemm_down(c, h->maps_dn, h->num_sms, st));
         pf.mark(5);
         CUDA_TRY(launch_finalize(c, st));
         pf.mark(6);
@@ -499,7 +548,13 @@ int moe_status(moe_handle* h) {
     uint32_t s = 0;
     CUDA_TRY(cudaMemcpy(&s, h->base.status, sizeof s, cudaMemcpyDeviceToHost));
     CUDA_TRY(cudaMemset(h->base.status, 0, sizeof s));
-    if (s & MOE_STATUS_TIMEOUT) return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
+    if (s & MOE_STATUS_TIMEOUT) {
+        // a kernel gave up part-way: put the fused decode's self-cleaning state back to zero
+        CUDA_TRY(cudaMemset(h->base.dfz.bar, 0, 2 * sizeof(unsigned)));
+        CUDA_TRY(cudaMemset(h->base.dfz.cnt, 0, sizeof(unsigned) * (size_t)(h->L.H / 32)));
+        CUDA_TRY(cudaMemset(h->base.dfz.outacc, 0, sizeof(float) * (size_t)h->L.H));
+        return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
+    }
     if (s & MOE_STATUS_BOUNDS) return fail(MOE_ERR_DEVICE_BOUNDS, "a device-side index check failed");
     if (s & MOE_STATUS_RANGE) return fail(MOE_ERR_RANGE, "a value exceeded the fp16 operand range");
     return MOE_OK;
@@ -512,7 +567,7 @@ int moe_debug_copy(moe_handle* h, int which, void* dst, size_t bytes, void* stre
     size_t cap = 0;
     switch (which) {
         case 0: src = h->base.act; cap = sizeof(__half) * (size_t)L.rows_cap * L.I; break;
-        case 1: src = h->base.xp; cap = sizeof(__half) * (size_t)L.rows_cap * L.H; break;
+        case 1: src = h->base.x16; cap = sizeof(__half) * (size_t)L.Tm * L.H; break;
         case 2: src = h->base.part; cap = sizeof(float) * (size_t)L.Tm * L.E; break;
         case 3: src = h->base.acc; cap = sizeof(float) * (size_t)L.Tm * L.H; break;
         default: return fail(MOE_ERR_INVALID_ARG, "unknown buffer %d", which);

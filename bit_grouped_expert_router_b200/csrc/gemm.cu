@@ -2,31 +2,45 @@
 //
 // "Perplexity Open-Sources Lily..." section "The optimizations follow the workload": the 4-bit
 // weights are reconstructed inside the grouped matrix multiplication rather than expanded into a
-// full weight array in memory.  Here that reconstruction lands in tensor memory: per pipeline
-// stage a bulk copy brings one 4608-byte block of packed codes + fp16 scale/bias (128 weight rows
-// x 64 input columns) into shared memory, four "transform" warps turn it into fp16 weights (exact
-// for this format, see common.cuh) and store them with tcgen05.st into a TMEM stage, and one
-// thread issues tcgen05.mma with the weights as the TMEM A operand and the tokens' activations as
-// the shared-memory B operand (TMA tile load, 128-byte swizzle).  Swap-AB: M = 128 weight rows,
-// N = up to 128 tokens of one expert, so experts with few tokens still fill the M dimension.
+// full weight array in memory.  Here one bulk copy brings four 4608-byte blocks of packed codes +
+// fp16 scale/bias (128 weight rows x 4 x 64 input columns) into shared memory, eight "transform"
+// warps turn each block into an fp16 tile (exact for this format, see common.cuh) written straight
+// into the tensor core's 128-byte-swizzled K-major operand layout, and one thread issues
+// tcgen05.mma with that tile as A and a TMA tile of the expert's token rows as B, accumulating in
+// tensor memory.  Swap-AB: M = 128 weight rows, N = up to 256 tokens of one expert, so experts with
+// few tokens still fill the M dimension.  The dequantised weights exist only in shared memory.
 //
-//   gate/up kernel : per tile (expert, 128 interleaved gate/up rows, <=128 tokens), K = H.
-//                    Epilogue: act = silu(G) * U (G and U of one column i sit 16 TMEM lanes apart
-//                    in the same warp, paired with one shuffle), fp16, staged in shared memory and
-//                    written to the expert's act rows (only the tile's valid tokens).
-//   down kernel    : per tile (expert, 128 output rows, <=128 tokens), K = I.
-//                    Epilogue: y * gate (routing gate, or sigmoid gate for the shared expert)
-//                    reduced with fp32 atomics (red.global.add) into the token's accumulator row.
+// Shaped by measurement on this part: every TMA operation costs an SM at least ~360 cycles
+// whatever its size, while big copies stream at ~90 B/clk.  So the weight blocks travel four
+// k-steps per copy, the token tile is a single box per k-step whose height (64/128/256 rows)
+// follows the tile's token count, and the three operand rings are sized separately:
+//   weight ring  kWS stages x kWB blocks   (producer -> transform)
+//   token ring   kBS stages x 256 x 64     (producer -> MMA)
+//   A ring       kAS stages x 128 x 64     (transform -> MMA)
 //
-// Warp roles (320 threads, one persistent CTA per SM, tiles taken round-robin from the device-
+//   gate/up kernel : per tile (expert, 128 interleaved gate/up rows, <=256 tokens), K = H.
+//                    B = the expert's bucketed fp16 token rows (the shared expert reads the fp16
+//                    activations directly: its rows are all tokens in order).  Epilogue:
+//                    act = silu(G) * U (G and U of one column i sit 16 TMEM lanes apart in the
+//                    same warp, paired with one shuffle), fp16, staged in shared memory and written
+//                    to the expert's act rows (only the tile's valid tokens).
+//   down kernel    : per tile (expert, 128 output rows, <=256 tokens), K = I.  B = act rows.
+//                    Epilogue: y * gate (routing gate, or sigmoid gate for the shared expert) added
+//                    into the token's fp32 accumulator row with coalesced red.global.add.f32 (a warp
+//                    covers 32 consecutive rows = 128 contiguous bytes of one token's row; L2 takes
+//                    such reductions at ~5 TB/s on this part, twice the rate of bulk reductions).
+//
+// Warp roles (576 threads, one persistent CTA per SM, tiles taken round-robin from the device-
 // built tile list so no tile count ever travels to the host):
-//   warp 0      TMA producer (one lane)
+//   warp 0      TMA producer (lane 0)
 //   warp 1      TMEM allocator + MMA issuer (one lane)
-//   warps 2-5   transform: dequantise a stage into TMEM (warp w owns TMEM lanes 32*(w%4)..+31)
-//   warps 6-9   epilogue: drain a TMEM accumulator (double-buffered, so it overlaps the next tile)
-// TMEM columns: [0,128) and [128,256) accumulators, [256, 256+32*kStages) fp16 A stages.
-// Every wait is bounded (common.cuh); on a timeout the roles unwind, the producer waits for its
-// copies in flight, the MMA thread waits for its MMAs, and warp 1 frees the TMEM.
+//   warps 2-9   transform: dequantise a block into the A ring (thread = row, half of 64 columns)
+//   warps 10-17 epilogue: drain a TMEM accumulator (double-buffered, so it overlaps the next tile;
+//               warp w reads TMEM lanes 32*(w%4)..+31, the two warps of a lane quarter take
+//               alternate 32-column chunks)
+// TMEM: two 256-column fp32 accumulators.  Every wait is bounded (common.cuh); on a timeout the
+// roles unwind, the producer waits for its copies in flight, the MMA thread waits for its MMAs,
+// and warp 1 frees the TMEM.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -34,43 +48,64 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kEpiWarps = 8;
+constexpr int kTransformWarps = 8;
+constexpr int kEpiWarp0 = 2 + kTransformWarps;
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = kBN;
-constexpr int kACol0 = 2 * kAccCols;
-static_assert(kACol0 + 32 * kStages <= kTmemCols, "TMEM budget");
-static_assert(kBN % 32 == 0 && kBN <= 256, "tile N");
+static_assert(2 * kAccCols <= kTmemCols, "TMEM budget");
+static_assert(kBN == 256, "token tile");
 
-constexpr int kBTileBytes = kBN * 128;  // kBN rows x 64 fp16
-constexpr int kOffB = 0;
-constexpr int kOffW = kOffB + kStages * kBTileBytes;
-constexpr int kOffStage = kOffW + kStages * kBlockBytes;
-constexpr int kStageBytes = kBN * 128;  // act staging: kBN rows x 64 fp16
+constexpr int kWB = 4;   // weight blocks per bulk copy
+constexpr int kWS = 2;   // weight ring stages
+constexpr int kBS = 3;   // token ring stages
+constexpr int kAS = 3;   // A ring stages
+
+constexpr int kATileBytes = 128 * 128;      // 128 weight rows x 64 fp16
+constexpr int kBTileBytes = kBN * 128;      // up to 256 token rows x 64 fp16
+constexpr int kWStageBytes = kWB * kBlockBytes;
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kAS * kATileBytes;
+constexpr int kOffW = kOffB + kBS * kBTileBytes;
+constexpr int kOffStage = kOffW + kWS * kWStageBytes;
+constexpr int kStageBytes = kBN * 128;      // gate/up: kBN x 64 fp16 act staging
 constexpr int kOffMeta = kOffStage + kStageBytes;
-constexpr int kMetaBytes = 2 * kBN * 8;  // [2 buffers][kBN] token + gate
+constexpr int kMetaBytes = 2 * kBN * 16;    // [2 buffers][kBN] row pointer + gate (+ pad)
 constexpr int kOffBar = kOffMeta + kMetaBytes;
-constexpr int kNumBars = 3 * kStages + 5;
+constexpr int kNumBars = 2 * (kWS + kBS + kAS) + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-static_assert(kOffW % 16 == 0 && kOffStage % 16 == 0 && kOffMeta % 16 == 0 && kOffBar % 8 == 0, "align");
+static_assert(kOffB % 1024 == 0 && kOffW % 16 == 0 && kOffStage % 16 == 0 && kOffMeta % 16 == 0 &&
+                  kOffBar % 8 == 0,
+              "align");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g * u / (1.f + __expf(-g)); }
 
+__device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c) {
+    return t.x >= 0 && t.x < c.G && t.y >= 0 && t.z > 0 && t.z <= kBN && t.y + t.z <= c.rows_cap;
+}
+
 template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const __grid_constant__ CUtensorMap tmB) {
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* asm_ = smem + kOffA;
     uint8_t* bsm = smem + kOffB;
     uint8_t* wsm = smem + kOffW;
     __half* stage = reinterpret_cast<__half*>(smem + kOffStage);
-    int* meta_tok = reinterpret_cast<int*>(smem + kOffMeta);
-    float* meta_gate = reinterpret_cast<float*>(smem + kOffMeta + 2 * kBN * 4);
+    float** meta_row = reinterpret_cast<float**>(smem + kOffMeta);
+    float* meta_gate = reinterpret_cast<float*>(smem + kOffMeta + 2 * kBN * 8);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* full = bars;                  // TMA data landed           (1 arrive + tx)
-    uint64_t* afull = bars + kStages;       // fp16 A stage in TMEM      (128 arrives)
-    uint64_t* empty = bars + 2 * kStages;   // MMAs of the stage done    (commit)
-    uint64_t* accfull = bars + 3 * kStages; // accumulator ready         (commit)
-    uint64_t* accempty = accfull + 2;       // accumulator drained       (128 arrives)
+    uint64_t* wfull = bars;                 // weight blocks landed      (1 arrive + tx)
+    uint64_t* wempty = wfull + kWS;         // weight blocks consumed    (256 arrives)
+    uint64_t* bfull = wempty + kWS;         // token tile landed         (1 arrive + tx)
+    uint64_t* bempty = bfull + kBS;         // token tile's MMAs done    (commit)
+    uint64_t* afull = bempty + kBS;         // fp16 A tile written       (256 arrives)
+    uint64_t* aempty = afull + kAS;         // A tile's MMAs done        (commit)
+    uint64_t* accfull = aempty + kAS;       // accumulator ready         (commit)
+    uint64_t* accempty = accfull + 2;       // accumulator drained       (256 arrives)
     uint64_t* drainbar = accfull + 4;       // MMA drain on abort        (commit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -81,19 +116,27 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
     const uint8_t* wbase = GATEUP ? c.w_gu : c.w_dn;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&afull[s], 128);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kWS; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], 32 * kTransformWarps);
+        }
+        for (int s = 0; s < kBS; ++s) {
+            mbar_init(&bfull[s], 1);
+            mbar_init(&bempty[s], 1);
+        }
+        for (int s = 0; s < kAS; ++s) {
+            mbar_init(&afull[s], 32 * kTransformWarps);
+            mbar_init(&aempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accfull[b], 1);
-            mbar_init(&accempty[b], 128);
+            mbar_init(&accempty[b], 32 * kEpiWarps);
         }
         mbar_init(drainbar, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmB);
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 3; ++j) prefetch_tmap(&maps.m[i][j]);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -108,61 +151,95 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
-        if (lane == 0 && !(c.flags & 0x100u)) {
-            uint32_t it = 0;
+        // Lane 0 waits for ring slots and issues the copies (the rest of the warp follows along).
+        if (!(c.flags & 0x100u)) {
+            const int shared_base = (GATEUP && c.has_shared) ? c.offsets[c.E] : 0;
+            uint32_t wit = 0, bit = 0;
+            int ws = 0, bs = 0;
+            uint32_t wph = 0, bph = 0;
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
                 const int mt = tau % MT;
-                if (tile.x < 0 || tile.x >= c.G || tile.y < 0 || tile.y + tile.z > c.rows_cap) continue;
+                if (!tile_ok(tile, c)) continue;
+                const int n_inst = max(16, ((tile.z + 15) / 16) * 16);
+                const int hsel = n_inst <= 64 ? 0 : (n_inst <= 128 ? 1 : 2);
+                const bool from_x = GATEUP && c.has_shared && tile.x == c.E;   // shared expert: token order
+                const CUtensorMap* map = &maps.m[from_x ? 1 : 0][hsel];
+                const int y = from_x ? tile.y - shared_base : tile.y;
+                const uint32_t b_bytes = (uint32_t)(64 << hsel) * 128;
                 const uint8_t* wsrc = wbase + ((size_t)tile.x * MT + mt) * KS * kBlockBytes;
-                for (int kc = 0; kc < KS; ++kc, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, c.status)) goto producer_done;
-                    mbar_arrive_expect_tx(&full[s], kBlockBytes + kBTileBytes);
-                    bulk_g2s(wsm + s * kBlockBytes, wsrc + (size_t)kc * kBlockBytes, kBlockBytes, &full[s]);
-                    tma_load_2d(bsm + s * kBTileBytes, &tmB, kc * 64, tile.y, &full[s]);
+                for (int kc = 0; kc < KS; ++kc) {
+                    int ok = 1;
+                    if (lane == 0) {
+                        if (kc % kWB == 0) {
+                            const int nb = min(kWB, KS - kc);
+                            ok = mbar_wait(&wempty[ws], wph ^ 1u, abort_flag, c.status) ? 1 : 0;
+                            if (ok) {
+                                mbar_arrive_expect_tx(&wfull[ws], (uint32_t)nb * kBlockBytes);
+                                bulk_g2s(wsm + ws * kWStageBytes, wsrc + (size_t)kc * kBlockBytes,
+                                         (uint32_t)nb * kBlockBytes, &wfull[ws]);
+                                ++wit;
+                                if (++ws == kWS) { ws = 0; wph ^= 1u; }
+                            }
+                        }
+                        if (ok) ok = mbar_wait(&bempty[bs], bph ^ 1u, abort_flag, c.status) ? 1 : 0;
+                        if (ok) {
+                            mbar_arrive_expect_tx(&bfull[bs], b_bytes);
+                            tma_load_2d(bsm + bs * kBTileBytes, map, kc * 64, y, &bfull[bs]);
+                            ++bit;
+                            if (++bs == kBS) { bs = 0; bph ^= 1u; }
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) goto producer_done;
                 }
             }
         producer_done:
             // every copy issued must land before the CTA may exit
-            const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0u;
-            for (uint32_t i = first; i < it; ++i) mbar_drain(&full[i % kStages], (i / kStages) & 1u);
+            if (lane == 0) {
+                for (uint32_t i = wit > (uint32_t)kWS ? wit - kWS : 0u; i < wit; ++i)
+                    mbar_drain(&wfull[i % kWS], (i / kWS) & 1u);
+                for (uint32_t i = bit > (uint32_t)kBS ? bit - kBS : 0u; i < bit; ++i)
+                    mbar_drain(&bfull[i % kBS], (i / kBS) & 1u);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            uint32_t it = 0, tl = 0;
+            uint32_t tl = 0;
+            int as = 0, bs = 0;
+            uint32_t aph = 0, bph = 0;
             bool issued = false;
-            for (int tau = blockIdx.x; tau < total; tau += gridDim.x, ++tl) {
+            const uint32_t a0 = smem_u32(asm_), b0 = smem_u32(bsm);
+            for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
-                if (tile.x < 0 || tile.x >= c.G || tile.y < 0 || tile.y + tile.z > c.rows_cap) {
+                if (!tile_ok(tile, c)) {
                     if (tau % MT == 0) set_status(c.status, MOE_STATUS_BOUNDS);
-                    --tl;
                     continue;
                 }
                 const int n_inst = max(16, ((tile.z + 15) / 16) * 16);
                 const uint32_t idesc = idesc_f16(128, n_inst, false);
-                const uint32_t ab = tl & 1u, aph = (tl >> 1) & 1u;
-                if (!mbar_wait(&accempty[ab], aph ^ 1u, abort_flag, c.status)) goto mma_done;
-                tc_fence_after();
+                const uint32_t ab = tl & 1u, acph = (tl >> 1) & 1u;
+                if (!mbar_wait(&accempty[ab], acph ^ 1u, abort_flag, c.status)) goto mma_done;
                 const uint32_t d_tmem = tmem + ab * kAccCols;
-                for (int kc = 0; kc < KS; ++kc, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
-                    if (!mbar_wait(&afull[s], ph, abort_flag, c.status)) goto mma_done;
-                    if (!mbar_wait(&full[s], ph, abort_flag, c.status)) goto mma_done;
+                for (int kc = 0; kc < KS; ++kc) {
+                    if (!mbar_wait(&afull[as], aph, abort_flag, c.status)) goto mma_done;
+                    if (!mbar_wait(&bfull[bs], bph, abort_flag, c.status)) goto mma_done;
                     tc_fence_after();
-                    const uint32_t b_addr = smem_u32(bsm + s * kBTileBytes);
+                    const uint32_t a_addr = a0 + as * kATileBytes, b_addr = b0 + bs * kBTileBytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        mma_ts(d_tmem, tmem + kACol0 + 32 * s + 8 * kk, sdesc_sw128(b_addr + 32 * kk), idesc,
+                        mma_ss(d_tmem, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
                                (kc | kk) != 0 ? 1u : 0u);
                     }
                     issued = true;
-                    tc_commit(&empty[s]);
+                    tc_commit(&aempty[as]);
+                    tc_commit(&bempty[bs]);
+                    if (++as == kAS) { as = 0; aph ^= 1u; }
+                    if (++bs == kBS) { bs = 0; bph ^= 1u; }
                 }
                 tc_commit(&accfull[ab]);
+                ++tl;
             }
         mma_done:
             if (*abort_flag && issued) {
@@ -170,66 +247,72 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                 mbar_drain(drainbar, 0);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------------ transform
-        const int q = warp & 3;
-        const int row = 32 * q + lane;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t it = 0;
+        // thread = (weight row, half of the 64 columns); the fp16 pairs of 16-byte chunk ch of row r
+        // go to r*128 + ((ch ^ (r & 7)) * 16), the 128-byte swizzle the MMA descriptor expects.
+        const int tt = threadIdx.x - 64;        // 0..255
+        const int row = tt & 127, half = tt >> 7;
+        const uint32_t sw = (uint32_t)(row & 7);
+        int ws = 0, as = 0;
+        uint32_t wph = 0, aph = 0;
         for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
             const int4 tile = c.tiles1[tau / MT];
-            if (tile.x < 0 || tile.x >= c.G || tile.y < 0 || tile.y + tile.z > c.rows_cap) continue;
-            for (int kc = 0; kc < KS; ++kc, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1u;
-                if (!mbar_wait(&full[s], ph, abort_flag, c.status)) goto transform_done;
-                const uint8_t* blk = wsm + s * kBlockBytes;
-                const uint4 c0 = *reinterpret_cast<const uint4*>(blk + row * 16);
-                const uint4 c1 = *reinterpret_cast<const uint4*>(blk + 2048 + row * 16);
+            if (!tile_ok(tile, c)) continue;
+            for (int kc = 0; kc < KS; ++kc) {
+                if (kc % kWB == 0 && !mbar_wait(&wfull[ws], wph, abort_flag, c.status)) goto transform_done;
+                if (!mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status)) goto transform_done;
+                const uint8_t* blk = wsm + ws * kWStageBytes + (kc % kWB) * kBlockBytes;
+                const uint4 cw = *reinterpret_cast<const uint4*>(blk + half * 2048 + row * 16);
                 const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
                 const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)),
                                            __ushort_as_half((unsigned short)(sb & 0xFFFFu)));
                 const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)),
                                            __ushort_as_half((unsigned short)(sb >> 16)));
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t r[32];
+                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint8_t* arow = asm_ + as * kATileBytes + row * 128;
 #pragma unroll
-                for (int w = 0; w < 8; ++w) {
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t r[4];
 #pragma unroll
                     for (int sft = 0; sft < 4; ++sft) {
                         const __half2 v = __hfma2(codes_to_half2(words[w], sft), s2, b2);
-                        r[4 * w + sft] = *reinterpret_cast<const uint32_t*>(&v);
+                        r[sft] = *reinterpret_cast<const uint32_t*>(&v);
                     }
+                    const uint32_t ch = (uint32_t)(4 * half + w);
+                    *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(r[0], r[1], r[2], r[3]);
                 }
-                tmem_st32(tmem + lane_base + kACol0 + 32 * s, r);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&afull[s]);
+                fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+                mbar_arrive(&afull[as]);
+                if (++as == kAS) { as = 0; aph ^= 1u; }
+                if (kc % kWB == kWB - 1 || kc == KS - 1) {   // this weight stage is used up
+                    mbar_arrive(&wempty[ws]);
+                    if (++ws == kWS) { ws = 0; wph ^= 1u; }
+                }
             }
         }
     transform_done:;
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;
-        const int etid = threadIdx.x - 192;
+        const int eh = (warp - kEpiWarp0) >> 2;           // which of the two warps of this quarter
+        const int etid = threadIdx.x - 32 * kEpiWarp0;   // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint32_t tl = 0;
         bool range_bad = false;
-        for (int tau = blockIdx.x; tau < total; tau += gridDim.x, ++tl) {
+        for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
             const int4 tile = c.tiles1[tau / MT];
             const int mt = tau % MT;
-            if (tile.x < 0 || tile.x >= c.G || tile.y < 0 || tile.y + tile.z > c.rows_cap) {
-                --tl;
-                continue;
-            }
+            if (!tile_ok(tile, c)) continue;
             const int row0 = tile.y, nvalid = tile.z;
             const uint32_t ab = tl & 1u, aph = (tl >> 1) & 1u;
+            ++tl;
             if (!GATEUP) {
-                if (etid < nvalid) {
-                    meta_tok[ab * kBN + etid] = c.row_token[row0 + etid];
-                    meta_gate[ab * kBN + etid] = c.row_gate[row0 + etid];
+                for (int j = etid; j < nvalid; j += 32 * kEpiWarps) {
+                    meta_row[ab * kBN + j] = c.acc + (size_t)c.row_token[row0 + j] * c.H + mt * 128;
+                    meta_gate[ab * kBN + j] = c.row_gate[row0 + j];
                 }
-                named_bar(1, 128);
+                named_bar(1, 32 * kEpiWarps);
             }
             if (!mbar_wait(&accfull[ab], aph, abort_flag, c.status)) goto epilogue_done;
             tc_fence_after();
@@ -237,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
             if (GATEUP) {
                 const int ilocal = 16 * q + (lane & 15);
                 const bool is_gate = lane < 16;
-                for (int c0 = 0; c0 < nvalid; c0 += 32) {
+                for (int c0 = 32 * eh; c0 < nvalid; c0 += 64) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
 #pragma unroll
@@ -255,28 +338,26 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                 }
                 tc_fence_before();
                 mbar_arrive(&accempty[ab]);
-                named_bar(1, 128);
+                named_bar(1, 32 * kEpiWarps);
                 const size_t I = (size_t)c.I;
-                for (int idx = etid; idx < nvalid * 8; idx += 128) {
+                for (int idx = etid; idx < nvalid * 8; idx += 32 * kEpiWarps) {
                     const int j = idx >> 3, ch = idx & 7;
                     *reinterpret_cast<uint4*>(c.act + (size_t)(row0 + j) * I + mt * 64 + ch * 8) =
                         *reinterpret_cast<const uint4*>(stage + j * 64 + ch * 8);
                 }
-                named_bar(1, 128);
+                named_bar(1, 32 * kEpiWarps);
             } else {
-                const int h = mt * 128 + 32 * q + lane;
-                float* accp = c.acc + h;
-                for (int c0 = 0; c0 < nvalid; c0 += 32) {
+                const int hl = 32 * q + lane;   // output row inside the m-tile
+                for (int c0 = 32 * eh; c0 < nvalid; c0 += 64) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
 #pragma unroll
                     for (int r = 0; r < 32; ++r) {
                         const int j = c0 + r;
                         if (j < nvalid) {
+                            float* dst = meta_row[ab * kBN + j] + hl;
                             const float y = __uint_as_float(v[r]) * meta_gate[ab * kBN + j];
-                            const int tok = meta_tok[ab * kBN + j];
-                            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(accp + (size_t)tok * c.H), "f"(y)
-                                         : "memory");
+                            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst), "f"(y) : "memory");
                         }
                     }
                 }
@@ -296,23 +377,46 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
     }
 }
 
+// xp[p] = x16[row_token[p]] for the T*k routed bucket rows: one warp per row, 16-byte copies.
+__global__ void __launch_bounds__(256) gather_rows_kernel(Ctx c) {
+    const int lane = lane_id();
+    const int nrows = c.T * c.k;
+    for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < nrows; p += gridDim.x * 8) {
+        const int t = c.row_token[p];
+        if (t < 0 || t >= c.T) {
+            if (lane == 0) set_status(c.status, MOE_STATUS_BOUNDS);
+            continue;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(c.x16 + (size_t)t * c.H);
+        uint4* dst = reinterpret_cast<uint4*>(c.xp + (size_t)p * c.H);
+        for (int i = lane; i < c.H / 8; i += 32) dst[i] = src[i];
+    }
+}
+
 }  // namespace
 
 int gemm_smem_bytes(bool) { return kSmemBytes; }
 
-cudaError_t launch_gemm_gateup(const Ctx& c, const CUtensorMap& tm_xp, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<true><<<num_sms, kThreads, kSmemBytes, st>>>(c, tm_xp);
+cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st) {
+    const int rows = c.T * c.k;
+    const int blocks = max(1, min((rows + 7) / 8, num_sms * 8));
+    gather_rows_kernel<<<blocks, 256, 0, st>>>(c);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_down(const Ctx& c, const CUtensorMap& tm_act, int num_sms, cudaStream_t st) {
+cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    grouped_gemm_kernel<true><<<num_sms, kThreads, kSmemBytes, st>>>(c, maps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<false><<<num_sms, kThreads, kSmemBytes, st>>>(c, tm_act);
+    grouped_gemm_kernel<false><<<num_sms, kThreads, kSmemBytes, st>>>(c, maps);
     return cudaGetLastError();
 }
 

@@ -9,8 +9,8 @@
 namespace moe {
 
 // Tile geometry of the prefill grouped GEMMs (tokens per tile = UMMA N).
-constexpr int kBN = 128;          // token columns per tile
-constexpr int kStages = 6;        // pipeline depth (smem stages == TMEM A-operand stages)
+constexpr int kBN = 256;          // token columns per tile (= UMMA N)
+constexpr int kStages = 3;        // pipeline depth (shared-memory stages)
 constexpr int kTokPerBucketBlk = 64;  // tokens per routing/bucketing CTA
 constexpr int kRouterTT = 32;     // tokens per CTA in the SIMT router (prefill sizes)
 constexpr int kRouterTTSmall = 8; // tokens per CTA in the SIMT router (decode sizes)
@@ -31,6 +31,16 @@ struct RepackArgs {
     uint32_t* inexact;
 };
 
+// Workspace of the fused batch-1 decode kernel.  outacc and cnt are zero between calls (the
+// kernel re-zeroes what it used); bar is the grid barrier {arrivals, generation}.
+struct DecodeFusedWs {
+    float* rpart;    // [4][E] quarter-row router partial logits
+    float* gu;       // [k+1][4][2I] gate/up k-range partial sums
+    float* outacc;   // [H] fp32 output accumulator
+    unsigned* cnt;   // [H/32] arrivals per 32-row output chunk
+    unsigned* bar;   // [2]
+};
+
 // Everything a forward-path kernel needs (passed by value).
 struct Ctx {
     int T, H, I, E, k, G, has_shared;
@@ -43,6 +53,7 @@ struct Ctx {
     const uint8_t* w_gu;
     const uint8_t* w_dn;
     const float* wrt;
+    const float* router32;   // router fp32 [E][H] (public layout copy)
     const float* rbias;
     const float* sgw;
     // call inputs / outputs
@@ -62,13 +73,15 @@ struct Ctx {
     int* perm;
     int* row_token;
     float* row_gate;
-    __half* xp;
+    __half* x16;      // [T][H] fp16 copy of the activations (prefill path)
+    __half* xp;       // [T*k][H] fp16 token rows in bucket order (routed experts)
     __half* act;
     float* acc;
     float* dact;
     float* dscale;
     uint32_t* status;
     unsigned int* counters;
+    DecodeFusedWs dfz;
 };
 
 cudaError_t launch_repack(const RepackArgs& a, int groups, int m_tiles, int k_steps, cudaStream_t st);
@@ -78,16 +91,25 @@ cudaError_t launch_router_prep(const float* router, const float* bias, const flo
 // routing + bucketing
 cudaError_t launch_router_simt(const Ctx& c, cudaStream_t st);
 cudaError_t launch_router_split(const float* router, int H, int E, int Epad, uint16_t* wsplit, cudaStream_t st);
-cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmA, const CUtensorMap& tmB, int mtiles,
+cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmW, const CUtensorMap& tmX, int n_exp,
                              cudaStream_t st);
 int router_tc_smem_bytes();
+int router_tc_splits();
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
 cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st);
 
+// Token-tile TMA maps of one grouped GEMM: m[source][h] with box {64 columns, 64 << h rows}.
+// gate/up: source 0 = bucketed rows xp, source 1 = the activations x16 (shared expert);
+// down: source 0 = act (source 1 unused).
+struct TokenMaps {
+    CUtensorMap m[2][3];
+};
+
 // prefill grouped GEMMs
-cudaError_t launch_gemm_gateup(const Ctx& c, const CUtensorMap& tm_xp, int num_sms, cudaStream_t st);
-cudaError_t launch_gemm_down(const Ctx& c, const CUtensorMap& tm_act, int num_sms, cudaStream_t st);
+cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st);
+cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st);
+cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st);
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st);
 int gemm_smem_bytes(bool gateup);
 
@@ -95,6 +117,8 @@ int gemm_smem_bytes(bool gateup);
 void set_last_error(const char* msg);
 
 // decode sparse GEMV
+cudaError_t launch_decode_fused(const Ctx& c, int num_sms, cudaStream_t st);
+int decode_fused_smem_bytes(int H, int I);
 cudaError_t launch_gemv_gateup(const Ctx& c, cudaStream_t st);
 cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st);
 

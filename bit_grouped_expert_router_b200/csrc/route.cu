@@ -6,12 +6,13 @@
 // workload" (routing kept on the GPU, no CPU synchronisation during the MoE work).
 //
 // Bucketing is a stable counting sort done in three passes:
-//   topk      : per CTA of 64 tokens, a histogram of its expert choices;
+//   topk      : per 64-token bucketing block, a histogram of its expert choices (global atomics);
 //   bucket_scan (one CTA): per-expert exclusive scan over the CTAs -> each CTA's base inside the
 //               bucket, bucket sizes, bucket offsets, and the tile list of the grouped GEMMs;
 //   scatter   : per CTA, ranks within the CTA in token order (warp match_any), giving every
-//               (token, slot) entry its row in the bucketed layout; copies the token's
-//               activations (bf16 -> fp16) into that row and into its shared-expert row.
+//               (token, slot) entry its row in the bucketed layout with its token and gate (the
+//               grouped GEMM gathers the token's activation row from there), and re-zeroes its
+//               histogram row for the next call.
 #include <float.h>
 
 #include "common.cuh"
@@ -78,104 +79,115 @@ cudaError_t launch_router_simt(const Ctx& c, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-// ---- top-k, renormalised softmax gates, shared gate, per-CTA histogram ------------------------
-// One warp per token; lane L holds experts L, L+32, ... (E <= 256).  Selection: k rounds of a
-// warp arg-max (ties -> lower expert index); NaN logits are treated as -inf so every selected
-// index is valid.  Gates: exp(l_j - l_max) / sum over the selected (softmax restricted to the
-// selection and renormalised).  Shared gate: sigmoid(x . w_sg).
+__device__ __forceinline__ uint32_t bf16x2_to_half2_bits(uint32_t w, bool* range_bad) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+    if (!(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f)) *range_bad = true;
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// ---- top-k, renormalised softmax gates, shared gate, bucket histogram ------------------------
+// One warp per token (8 per CTA); lane L holds experts L, L+32, ... (E <= 256), each the sum of the
+// c.ks partial logits plus the bias.  Selection: k rounds of a warp arg-max (ties -> lower expert
+// index); NaN logits are treated as -inf so every selected index is valid.  Gates:
+// exp(l_j - l_max) / sum over the selected (softmax restricted to the selection, renormalised).
+// Shared gate: sigmoid(x . w_sg).  Prefill path (do_hist): count the token's experts into the
+// histogram row of its 64-token bucketing block (global atomics; the scatter kernel re-zeroes the
+// row after use) and zero the token's fp32 accumulator row for the down-projection combine.
 __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
-    __shared__ int hist[256];
-    __shared__ float lg[8][256];
-    const int lane = lane_id(), warp = threadIdx.x >> 5;
-    if (do_hist) {
-        for (int e = threadIdx.x; e < c.E; e += blockDim.x) hist[e] = 0;
-    }
-    const int t_begin = blockIdx.x * kTokPerBucketBlk;
-    const int t_end = min(c.T, t_begin + kTokPerBucketBlk);
-    for (int tb = t_begin; tb < t_end; tb += 8) {
-        // phase 1: the block reduces the split-K partial logits of 8 tokens in parallel
-        __syncthreads();
-        for (int i = threadIdx.x; i < 8 * c.E; i += blockDim.x) {
-            const int tt = i / c.E, e = i % c.E;
-            const int t = tb + tt;
-            if (t < t_end) {
-                float s = 0.f;
-#pragma unroll 8
-                for (int q = 0; q < c.ks; ++q) s += c.part[((size_t)q * c.T + t) * c.E + e];
-                s += c.rbias[e];
-                lg[tt][e] = (s != s) ? -INFINITY : s;
-            }
+    const int lane = lane_id();
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= c.T) return;
+    float l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        float v = -INFINITY;
+        if (e < c.E) {
+            float s = 0.f;
+            for (int q = 0; q < c.ks; ++q) s += c.part[((size_t)q * c.T + t) * c.E + e];
+            s += c.rbias[e];
+            v = (s != s) ? -INFINITY : s;
         }
-        __syncthreads();
-        // phase 2: one warp per token selects the top k
-        const int t = tb + warp;
-        if (t >= t_end) continue;
-        float l[8];
+        l[i] = v;
+    }
+    unsigned taken = 0;
+    int my_e = 0;
+    float my_v = 0.f;
+    for (int j = 0; j < c.k; ++j) {
+        float bv = 0.f;
+        int be = 0x7fffffff;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int e = lane + 32 * i;
-            l[i] = (e < c.E) ? lg[warp][e] : -INFINITY;
-        }
-        unsigned taken = 0;
-        int my_e = 0;
-        float my_v = 0.f;
-        for (int j = 0; j < c.k; ++j) {
-            float bv = 0.f;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                if (e < c.E && !((taken >> i) & 1u)) {
-                    if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
-                }
+            if (e < c.E && !((taken >> i) & 1u)) {
+                if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            if (lane == j) { my_e = be; my_v = bv; }
         }
-        const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-        const float p = (lane < c.k) ? expf(my_v - vmax) : 0.f;
-        float z = p;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-        if (lane < c.k) {
-            if (my_e < 0 || my_e >= c.E) { set_status(c.status, MOE_STATUS_BOUNDS); my_e = 0; }
-            c.idx[(size_t)t * c.k + lane] = my_e;
-            c.gates[(size_t)t * c.k + lane] = p / z;
-            if (do_hist) atomicAdd(&hist[my_e], 1);
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
         }
-        float sgv = 0.f;
-        if (c.has_shared) {
-            float d = 0.f;
-            const uint16_t* xr = c.x + (size_t)t * c.H;
-            for (int h = lane * 8; h < c.H; h += 256) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(xr + h);
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    d = fmaf(__uint_as_float(w4[q] << 16), c.sgw[h + 2 * q], d);
-                    d = fmaf(__uint_as_float(w4[q] & 0xFFFF0000u), c.sgw[h + 2 * q + 1], d);
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            sgv = 1.f / (1.f + expf(-d));
-        }
-        if (lane == 0) c.sg[t] = sgv;
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) { my_e = be; my_v = bv; }
     }
+    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const float p = (lane < c.k) ? expf(my_v - vmax) : 0.f;
+    float z = p;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane < c.k) {
+        if (my_e < 0 || my_e >= c.E) { set_status(c.status, MOE_STATUS_BOUNDS); my_e = 0; }
+        c.idx[(size_t)t * c.k + lane] = my_e;
+        c.gates[(size_t)t * c.k + lane] = p / z;
+        if (do_hist) atomicAdd(&c.hist[(size_t)(t / kTokPerBucketBlk) * c.E + my_e], 1);
+    }
+    float sgv = 0.f;
+    const uint16_t* xr = c.x + (size_t)t * c.H;
+    float d = 0.f;
+    bool range_bad = false;
+    if (c.has_shared || do_hist) {
+        for (int h = lane * 8; h < c.H; h += 256) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(xr + h);
+            if (c.has_shared) {
+                const float4 w0 = *reinterpret_cast<const float4*>(c.sgw + h);
+                const float4 w1 = *reinterpret_cast<const float4*>(c.sgw + h + 4);
+                d = fmaf(__uint_as_float(raw.x << 16), w0.x, d);
+                d = fmaf(__uint_as_float(raw.x & 0xFFFF0000u), w0.y, d);
+                d = fmaf(__uint_as_float(raw.y << 16), w0.z, d);
+                d = fmaf(__uint_as_float(raw.y & 0xFFFF0000u), w0.w, d);
+                d = fmaf(__uint_as_float(raw.z << 16), w1.x, d);
+                d = fmaf(__uint_as_float(raw.z & 0xFFFF0000u), w1.y, d);
+                d = fmaf(__uint_as_float(raw.w << 16), w1.z, d);
+                d = fmaf(__uint_as_float(raw.w & 0xFFFF0000u), w1.w, d);
+            }
+            if (do_hist) {   // fp16 copy of the row for the tensor-core path (exact for |x| < 65504)
+                uint4 o;
+                o.x = bf16x2_to_half2_bits(raw.x, &range_bad);
+                o.y = bf16x2_to_half2_bits(raw.y, &range_bad);
+                o.z = bf16x2_to_half2_bits(raw.z, &range_bad);
+                o.w = bf16x2_to_half2_bits(raw.w, &range_bad);
+                *reinterpret_cast<uint4*>(c.x16 + (size_t)t * c.H + h) = o;
+            }
+        }
+    }
+    if (c.has_shared) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        sgv = 1.f / (1.f + expf(-d));
+    }
+    if (range_bad) set_status(c.status, MOE_STATUS_RANGE);
+    if (lane == 0) c.sg[t] = sgv;
     if (do_hist) {
-        __syncthreads();
-        for (int e = threadIdx.x; e < c.E; e += blockDim.x) c.hist[(size_t)blockIdx.x * c.E + e] = hist[e];
+        float4* ar = reinterpret_cast<float4*>(c.acc + (size_t)t * c.H);
+        for (int h4 = lane; h4 < c.H / 4; h4 += 32) ar[h4] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st) {
-    topk_kernel<<<c.nblk, 256, 0, st>>>(c, histogram ? 1 : 0);
+    topk_kernel<<<(c.T + 7) / 8, 256, 0, st>>>(c, histogram ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -190,17 +202,41 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
     return v;
 }
 
+// Four threads per expert each scan a quarter of the bucketing blocks (loads issued eight at a
+// time), the quarters are combined in shared memory, and a second pass writes every block's base
+// inside each bucket back into the histogram rows.
 __global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
+    __shared__ int part[4][256];
     __shared__ int cnt[264], off[264], toff[264];
     const int tid = threadIdx.x, lane = lane_id();
-    for (int e = tid; e < c.E; e += blockDim.x) {
-        int run = 0;
-        for (int b = 0; b < c.nblk; ++b) {
-            const int v = c.hist[(size_t)b * c.E + e];
-            c.hist[(size_t)b * c.E + e] = run;  // becomes this CTA's base inside bucket e
-            run += v;
+    const int e = tid & 255, quarter = tid >> 8;
+    const int b_lo = quarter * c.nblk / 4, b_hi = (quarter + 1) * c.nblk / 4;
+    int sum = 0;
+    if (e < c.E) {
+        for (int b0 = b_lo; b0 < b_hi; b0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = (b0 + u < b_hi) ? c.hist[(size_t)(b0 + u) * c.E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sum += v[u];
         }
-        cnt[e] = run;
+    }
+    part[quarter][e] = sum;
+    __syncthreads();
+    if (e < c.E) {
+        int run = 0;
+        for (int qq = 0; qq < quarter; ++qq) run += part[qq][e];
+        if (quarter == 3) cnt[e] = run + sum;
+        for (int b0 = b_lo; b0 < b_hi; b0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = (b0 + u < b_hi) ? c.hist[(size_t)(b0 + u) * c.E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (b0 + u < b_hi) c.hist[(size_t)(b0 + u) * c.E + e] = run;  // block base inside bucket e
+                run += v[u];
+            }
+        }
     }
     if (tid == 0 && c.has_shared) cnt[c.E] = c.T;
     __syncthreads();
@@ -240,23 +276,18 @@ cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-// ---- scatter: bucket positions, row metadata, gathered fp16 activations ------------------------
-__device__ __forceinline__ uint32_t bf16x2_to_half2_bits(uint32_t w, bool* range_bad) {
-    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
-    if (!(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f)) *range_bad = true;
-    const __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
+// ---- scatter: bucket positions and row metadata ---------------------------------------------
 
 __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
     extern __shared__ int sm[];
     int* cnt = sm;          // [E] next free row of each bucket for this CTA
-    int* pos = sm + c.E;    // [64 * k] row of each (token, slot) of this CTA
     const int lane = lane_id(), warp = threadIdx.x >> 5;
     const int t0 = blockIdx.x * kTokPerBucketBlk;
     const int nt = min(kTokPerBucketBlk, c.T - t0);
-    for (int e = threadIdx.x; e < c.E; e += blockDim.x)
+    for (int e = threadIdx.x; e < c.E; e += blockDim.x) {
         cnt[e] = c.offsets[e] + c.hist[(size_t)blockIdx.x * c.E + e];
+        c.hist[(size_t)blockIdx.x * c.E + e] = 0;   // ready for the next call's counting
+    }
     __syncthreads();
     if (warp == 0) {
         const int n_entries = nt * c.k;
@@ -275,9 +306,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
             if (active) {
                 if (p < 0 || p >= c.rows_cap) {
                     set_status(c.status, MOE_STATUS_BOUNDS);
-                    pos[i] = -1;
                 } else {
-                    pos[i] = p;
                     c.perm[p] = flat;
                     c.row_token[p] = flat / c.k;
                     c.row_gate[p] = c.gates[flat];
@@ -287,35 +316,17 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
     }
     __syncthreads();
     const int shared_base = c.offsets[c.E];
-    bool range_bad = false;
-    for (int tt = warp; tt < nt; tt += 8) {
-        const int t = t0 + tt;
-        const uint16_t* xr = c.x + (size_t)t * c.H;
-        for (int h = lane * 8; h < c.H; h += 256) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(xr + h);
-            uint4 o;
-            o.x = bf16x2_to_half2_bits(raw.x, &range_bad);
-            o.y = bf16x2_to_half2_bits(raw.y, &range_bad);
-            o.z = bf16x2_to_half2_bits(raw.z, &range_bad);
-            o.w = bf16x2_to_half2_bits(raw.w, &range_bad);
-            for (int j = 0; j < c.k; ++j) {
-                const int p = pos[tt * c.k + j];
-                if (p >= 0) *reinterpret_cast<uint4*>(c.xp + (size_t)p * c.H + h) = o;
-            }
-            if (c.has_shared) *reinterpret_cast<uint4*>(c.xp + (size_t)(shared_base + t) * c.H + h) = o;
-        }
-        float4* ar = reinterpret_cast<float4*>(c.acc + (size_t)t * c.H);
-        for (int h4 = lane; h4 < c.H / 4; h4 += 32) ar[h4] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c.has_shared && lane == 0) {
+    if (c.has_shared) {
+        for (int tt = threadIdx.x; tt < nt; tt += blockDim.x) {
+            const int t = t0 + tt;
             c.row_token[shared_base + t] = t;
             c.row_gate[shared_base + t] = c.sg[t];
         }
     }
-    if (range_bad) set_status(c.status, MOE_STATUS_RANGE);
 }
 
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st) {
-    const size_t smem = sizeof(int) * (size_t)(c.E + kTokPerBucketBlk * c.k);
+    const size_t smem = sizeof(int) * (size_t)c.E;
     scatter_kernel<<<c.nblk, 256, smem, st>>>(c);
     return cudaGetLastError();
 }

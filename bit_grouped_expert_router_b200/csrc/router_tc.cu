@@ -1,16 +1,19 @@
 // router_tc.cu -- prefill router logits on the tensor core.
 //
 // logits[t][e] = sum_h x[t][h] * W[e][h] with W the fp32 router.  W is split once (at create) into
-// two bf16 terms, Wh = bf16(W) and Wl = bf16(W - Wh), which together carry 16 significant bits of
-// each weight (relative residual <= 2^-16); x is bf16 already, so every product x*Wh and x*Wl is
-// exact in the fp32 accumulator and the GEMM over K = 2H of [Wh | Wl] against [x | x] reproduces
-// the fp32 dot product to a few 1e-6 -- far inside the 1e-3 top-(k+1) logit gap the routing is
-// checked with.  (The split-K SIMT router in route.cu stays in use for decode-sized T.)
+// two bf16 terms, W1 = bf16(W) and W2 = bf16(W - W1), which carry 16 significant bits of every
+// weight (relative residual <= 2^-17); x is bf16 already, so every product x*Wi is exact.  The
+// tensor core's fp32 accumulation does not round to nearest on every add, so long accumulation
+// chains drift: the K = 2H products of one logit are split four ways into separate partial sums
+// (each its own short chain on the tensor core) that the top-k kernel adds in fp32.  Measured
+// against the fp64 oracle the logits agree to a few 1e-6 -- far inside the 1e-3 top-(k+1) gap
+// the routing is checked with.  (The split-K SIMT router in route.cu serves decode-sized T.)
 //
-// One CTA per 64 tokens computes all experts (two 128-row m-tiles for E = 256): TMA brings the
-// 128x64 bf16 tiles of [Wh | Wl] and the 64x64 tile of x (128-byte swizzle) into a 4-stage ring,
-// one thread issues tcgen05.mma (both operands in shared memory, fp32 accumulators in TMEM), and
-// four epilogue warps write the raw logits [T][E] (fp32) for the top-k kernel.
+// CTA (token tile of 128, K quarter): TMA brings the 128x64 bf16 tile of x (A, M = 128 tokens) and
+// the Epad16x64 tile of [W1 | W2] (B, N = all experts, <= 256) into a 4-stage ring with the
+// 128-byte swizzle; one thread issues tcgen05.mma (both operands in shared memory, fp32
+// accumulator in TMEM, lane = token, column = expert); four epilogue warps write the partial
+// logits part[quarter][t][e] with 16-byte stores (a thread owns one token's row).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,17 +21,18 @@ namespace moe {
 
 namespace {
 
-constexpr int kRN = 64;        // tokens per CTA (UMMA N)
+constexpr int kRM = 128;        // tokens per CTA (UMMA M)
+constexpr int kRSplit = 4;      // K quarters (partial sums)
 constexpr int kRStages = 4;
 constexpr int kRThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
-constexpr int kRAT = 128 * 128;  // bytes of one 128-row x 64-col bf16 A tile
-constexpr int kRBT = kRN * 128;  // bytes of the B tile
-constexpr int kRStageBytes = 2 * kRAT + kRBT;
+constexpr int kRAT = kRM * 128;  // bytes of the x tile
+constexpr int kRBTMax = 256 * 128;
+constexpr int kRStageBytes = kRAT + kRBTMax;
 constexpr int kROffBar = kRStages * kRStageBytes;
 constexpr int kRSmem = kROffBar + (2 * kRStages + 2) * 8 + 16 + 1024;
 
 __global__ void __launch_bounds__(kRThreads, 1)
-    router_tc_kernel(Ctx c, int mtiles, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB) {
+    router_tc_kernel(Ctx c, int n_exp, const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kROffBar);
@@ -39,10 +43,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = lane_id();
-    const int t0 = blockIdx.x * kRN;
-    const int nvalid = min(kRN, c.T - t0);
-    const int KH = c.H / 64;     // k-steps per half (x tile repeats in the second half)
+    const int t0 = blockIdx.x * kRM;
+    const int split = blockIdx.y;
+    const int KH = c.H / 64;                 // k-steps per term (the x tile repeats for each term)
     const int KS = 2 * KH;
+    const int k_begin = split * KS / kRSplit, k_end = (split + 1) * KS / kRSplit;
+    const int tmem_cols = n_exp <= 32 ? 32 : (n_exp <= 64 ? 64 : (n_exp <= 128 ? 128 : 256));
+    const uint32_t b_bytes = (uint32_t)n_exp * 128;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRStages; ++s) {
@@ -53,11 +60,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
         mbar_init(drainbar, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmW);
+        prefetch_tmap(&tmX);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 2 * kRN);
+        tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -68,37 +75,33 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             uint32_t it = 0;
-            for (int kc = 0; kc < KS; ++kc, ++it) {
+            for (int kc = k_begin; kc < k_end; ++kc, ++it) {
                 const int s = it % kRStages;
                 const uint32_t ph = (it / kRStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, c.status)) break;
                 uint8_t* st = smem + s * kRStageBytes;
-                mbar_arrive_expect_tx(&full[s], mtiles * kRAT + kRBT);
-                for (int mt = 0; mt < mtiles; ++mt) tma_load_2d(st + mt * kRAT, &tmA, kc * 64, mt * 128, &full[s]);
-                tma_load_2d(st + 2 * kRAT, &tmB, (kc % KH) * 64, t0, &full[s]);
+                mbar_arrive_expect_tx(&full[s], kRAT + b_bytes);
+                tma_load_2d(st, &tmX, (kc % KH) * 64, t0, &full[s]);
+                tma_load_2d(st + kRAT, &tmW, kc * 64, 0, &full[s]);
             }
             const uint32_t first = it > (uint32_t)kRStages ? it - kRStages : 0u;
             for (uint32_t i = first; i < it; ++i) mbar_drain(&full[i % kRStages], (i / kRStages) & 1u);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const int n_inst = max(16, ((nvalid + 15) / 16) * 16);
-            const uint32_t idesc = idesc_f16(128, n_inst, true);
+            const uint32_t idesc = idesc_f16(kRM, n_exp, true);
             bool ok = true, issued = false;
             uint32_t it = 0;
-            for (int kc = 0; kc < KS; ++kc, ++it) {
+            for (int kc = k_begin; kc < k_end; ++kc, ++it) {
                 const int s = it % kRStages;
                 const uint32_t ph = (it / kRStages) & 1u;
                 if (!mbar_wait(&full[s], ph, abort_flag, c.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + s * kRStageBytes);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = sdesc_sw128(st + 2 * kRAT + 32 * kk);
-                    for (int mt = 0; mt < mtiles; ++mt)
-                        mma_ss(tmem + mt * kRN, sdesc_sw128(st + mt * kRAT + 32 * kk), bdesc, idesc,
-                               (kc | kk) != 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem, sdesc_sw128(st + 32 * kk), sdesc_sw128(st + kRAT + 32 * kk), idesc,
+                           (kc != k_begin || kk) ? 1u : 0u);
                 issued = true;
                 tc_commit(&empty[s]);
             }
@@ -110,19 +113,24 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
     } else {
         const int q = warp & 3;
+        const int t = t0 + 32 * q + lane;
         if (mbar_wait(accfull, 0, abort_flag, c.status)) {
             tc_fence_after();
-            for (int mt = 0; mt < mtiles; ++mt) {
-                const int e = mt * 128 + 32 * q + lane;
-                for (int c0 = 0; c0 < nvalid; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + mt * kRN + c0, v);
-                    if (e < c.E) {
+            float* dst = c.part + ((size_t)split * c.T + t) * c.E;
+            for (int c0 = 0; c0 < n_exp; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + c0, v);
+                if (t < c.T) {
+                    if (c0 + 32 <= c.E && (c.E & 3) == 0) {
 #pragma unroll
-                        for (int r = 0; r < 32; ++r) {
-                            const int j = c0 + r;
-                            if (j < nvalid) c.part[(size_t)(t0 + j) * c.E + e] = __uint_as_float(v[r]);
-                        }
+                        for (int r = 0; r < 32; r += 4)
+                            *reinterpret_cast<float4*>(dst + c0 + r) =
+                                make_float4(__uint_as_float(v[r]), __uint_as_float(v[r + 1]),
+                                            __uint_as_float(v[r + 2]), __uint_as_float(v[r + 3]));
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            if (c0 + r < c.E) dst[c0 + r] = __uint_as_float(v[r]);
                     }
                 }
             }
@@ -132,11 +140,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * kRN);
+        tmem_dealloc(tmem, tmem_cols);
     }
 }
 
-// Wsplit[e][h] = bf16(W[e][h]), Wsplit[e][H + h] = bf16(W[e][h] - that); rows e >= E are zero.
+// Wsplit[e][t*H + h] = term t of W[e][h] (t = 0, 1; the second is the bf16 rounding of what the
+// first left); rows e >= E are zero.
 __global__ void router_split_kernel(const float* __restrict__ router, int H, int E, int Epad,
                                     uint16_t* __restrict__ wsplit) {
     const size_t n = (size_t)Epad * H;
@@ -153,18 +162,20 @@ __global__ void router_split_kernel(const float* __restrict__ router, int H, int
 }  // namespace
 
 int router_tc_smem_bytes() { return kRSmem; }
+int router_tc_splits() { return kRSplit; }
 
 cudaError_t launch_router_split(const float* router, int H, int E, int Epad, uint16_t* wsplit, cudaStream_t st) {
     router_split_kernel<<<256, 256, 0, st>>>(router, H, E, Epad, wsplit);
     return cudaGetLastError();
 }
 
-cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmA, const CUtensorMap& tmB, int mtiles,
+// tmW: [W1 | W2] bf16 [Epad][2H], box {64, n_exp}; tmX: x bf16 [T][H], box {64, 128}.
+cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmW, const CUtensorMap& tmX, int n_exp,
                              cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
     if (e != cudaSuccess) return e;
-    const int blocks = (c.T + kRN - 1) / kRN;
-    router_tc_kernel<<<blocks, kRThreads, kRSmem, st>>>(c, mtiles, tmA, tmB);
+    dim3 grid((c.T + kRM - 1) / kRM, kRSplit);
+    router_tc_kernel<<<grid, kRThreads, kRSmem, st>>>(c, n_exp, tmW, tmX);
     return cudaGetLastError();
 }
 

@@ -70,6 +70,8 @@ extern "C" {
 
 /* ---- configuration flags ---------------------------------------------------------------------- */
 #define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
+#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* T == 1: use the multi-kernel GEMV chain instead of the
+                                          single cooperative decode kernel */
 #define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its first load,
                                           so the consumers' bounded waits run out and the call
                                           reports MOE_ERR_DEVICE_TIMEOUT; nothing traps or hangs */
@@ -148,7 +150,7 @@ MOE_API int moe_status(moe_handle *h);
 
 /* Debug: copy `bytes` of an internal workspace buffer to a caller device buffer (stream-ordered).
  * which: 0 = expert activations act[rows, I] (fp16, bucket order, prefill path),
- *        1 = gathered input rows xp[rows, H] (fp16, bucket order),
+ *        1 = fp16 copy of the activations x16[T, H] (prefill path),
  *        2 = router logits [T, E] (fp32, tensor-core router only),
  *        3 = fp32 combine accumulator [T, H].
  * Errors: INVALID_ARG when `which` is unknown or `bytes` exceeds the buffer. */
@@ -161,9 +163,10 @@ MOE_API int moe_debug_copy(moe_handle *h, int which, void *dst, size_t bytes, vo
  * device time in milliseconds (ms[MOE_PROF_SLOTS]) and the number of launches
  * (launches[MOE_PROF_SLOTS]), and clears the record.  Slots: 0 router logits, 1 top-k and gates,
  * 2 bucket scan, 3 scatter/gather, 4 gate/up grouped GEMM, 5 down grouped GEMM + combine,
- * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine.
+ * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine, 9 fused batch-1 decode (the
+ * whole layer in one kernel), 10 gather of token rows into bucket order.
  * Errors: INVALID_ARG, CUDA. */
-#define MOE_PROF_SLOTS 9
+#define MOE_PROF_SLOTS 11
 MOE_API int moe_profile_enable(moe_handle *h, int enable);
 MOE_API int moe_profile_read(moe_handle *h, float *ms, int32_t *launches);
 

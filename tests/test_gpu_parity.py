@@ -209,3 +209,50 @@ def test_fp16_range_overflow_is_reported():
     assert layer.status() == M.MOE_ERR_RANGE
     assert layer.status() == M.MOE_OK   # cleared
     layer.close()
+
+
+# ---------------------------------------------------------------------------------------------
+# batch-1 decode: the single cooperative kernel, the multi-kernel chain, and graph replay
+def test_decode_fused_and_unfused_agree_and_replay_in_a_graph():
+    shape = synth.WORKLOADS["decode"]
+    layers, xs, refs = [], [], []
+    for l in (0, 1):
+        w = synth.make_layer(shape, l)
+        ol = oracle.OracleLayer.from_shape(w, shape)
+        x = gapped_x(shape, ol, l, 0, T=1)
+        refs.append(ol.forward(x))
+        xs.append(x.cuda())
+        wc = _cuda(w)
+        layers.append((M.Layer.from_shape(wc, shape, max_tokens=16, decode_max_tokens=16),
+                       M.Layer.from_shape(wc, shape, max_tokens=16, decode_max_tokens=16,
+                                          flags=M.MOE_FLAG_DECODE_UNFUSED)))
+    for (fused, unfused), x, ref in zip(layers, xs, refs):
+        a = fused.forward(x)
+        b = unfused.forward(x)
+        torch.cuda.synchronize()
+        assert fused.status() == M.MOE_OK and unfused.status() == M.MOE_OK
+        compare(a.cpu(), ref)
+        compare(b.cpu(), ref)
+        # repeated calls reuse the self-cleaning accumulator state
+        for _ in range(3):
+            a2 = fused.forward(x)
+        torch.cuda.synchronize()
+        compare(a2.cpu(), ref)
+    # the fused kernels of two layers captured in one CUDA graph and replayed
+    outs = [torch.empty((1, shape.H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for (fused, _), x, o in zip(layers, xs, outs):
+            fused.forward(x, out=o)
+    for _ in range(5):
+        g.replay()
+    torch.cuda.synchronize()
+    for o, ref in zip(outs, refs):
+        compare(o.cpu(), ref)
+    del g
+    for f, u in layers:
+        assert f.status() == M.MOE_OK
+        f.close()
+        u.close()
