@@ -445,7 +445,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.dfz.bar = reinterpret_cast<unsigned*>(ws + L.o_dfz_bar);
 
     for (int hs = 0; hs < 3 && rc == MOE_OK; ++hs) {
-        const int box = 64 << hs;
+        const int box = 64 << hs;   // token tile box: 64, 128 or 256 rows
         rc = encode_rows_map(&h->maps_gu.m[0][hs], c.xp, L.Tm * L.k, L.H, box);
         if (rc == MOE_OK) rc = encode_rows_map(&h->maps_gu.m[1][hs], c.x16, L.Tm, L.H, box);
         if (rc == MOE_OK) rc = encode_rows_map(&h->maps_dn.m[0][hs], c.act, L.rows_cap, L.I, box);

@@ -16,8 +16,12 @@
 //            a 32-row chunk (atomic counter) rounds it to bf16, writes the output and re-zeroes the
 //            accumulator and counter for the next call (self-cleaning, no memset launch).
 //
-// Each phase is a flat list of warp tasks (one weight-block slice each) handed out by global warp
-// id, so all of a phase's weight loads are in flight at once.  GEMV arithmetic as in decode.cu.
+// Each phase is a flat list of warp tasks (one weight-block slice each); task t runs on CTA
+// t % grid, so every SM carries a share and all of a phase's weight loads are in flight at once.
+// The down blocks of phase 2 are requested into L2 early (bulk L2 prefetch: the shared expert's
+// at kernel start, the routed experts' right after top-k), and each phase-2 warp issues its
+// weight loads before it builds act, so phase 2 mostly waits on L2, not HBM.  GEMV arithmetic as
+// in decode.cu.
 // Grid barrier: arrival counter + generation word in the workspace; waits are bounded (1 s), on a
 // timeout the status word records it and moe_status resets the barrier state.
 #include "common.cuh"
@@ -107,33 +111,58 @@ struct GemvTask {  // one warp: 32 rows (lane = row) of one m-tile, k-steps [k0,
     int k0, k1;
 };
 
-__device__ __forceinline__ float run_gemv(const GemvTask& t, const float* vperm, const float* vsum, const float* vsc) {
-    // issue every load of the task first, then the arithmetic
-    constexpr int kMax = 8;
-    uint4 a[kMax], b[kMax];
-    uint32_t sb[kMax];
+// A task's codes and scale/bias words, loaded ahead of the arithmetic (up to 8 k-steps).
+struct GemvRegs {
+    uint4 a[8], b[8];
+    uint32_t sb[8];
+};
+
+__device__ __forceinline__ void gemv_load(const GemvTask& t, GemvRegs& r) {
     const int n = t.k1 - t.k0;
 #pragma unroll
-    for (int i = 0; i < kMax; ++i) {
+    for (int i = 0; i < 8; ++i) {
         if (i < n) {
             const uint8_t* blk = t.blocks + (size_t)(t.k0 + i) * kBlockBytes;
-            a[i] = __ldg(reinterpret_cast<const uint4*>(blk + t.row * 16));
-            b[i] = __ldg(reinterpret_cast<const uint4*>(blk + 2048 + t.row * 16));
-            sb[i] = __ldg(reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + t.row * 4));
+            r.a[i] = __ldg(reinterpret_cast<const uint4*>(blk + t.row * 16));
+            r.b[i] = __ldg(reinterpret_cast<const uint4*>(blk + 2048 + t.row * 16));
+            r.sb[i] = __ldg(reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + t.row * 4));
         }
     }
+}
+
+__device__ __forceinline__ float gemv_dot(const GemvTask& t, const GemvRegs& r, const float* vperm,
+                                          const float* vsum, const float* vsc) {
+    const int n = t.k1 - t.k0;
     float acc = 0.f;
 #pragma unroll
-    for (int i = 0; i < kMax; ++i) {
+    for (int i = 0; i < 8; ++i) {
         if (i < n) {
             const int cc = t.k0 + i;
-            const float s = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
-            const float bb = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
-            const float P = dot_group(a[i], b[i], vperm + 64 * cc);
+            const float s = __half2float(__ushort_as_half((unsigned short)(r.sb[i] & 0xFFFFu)));
+            const float bb = __half2float(__ushort_as_half((unsigned short)(r.sb[i] >> 16)));
+            const float P = dot_group(r.a[i], r.b[i], vperm + 64 * cc);
             acc += s * (P * vsc[cc]) + bb * vsum[cc];
         }
     }
     return acc;
+}
+
+__device__ __forceinline__ float run_gemv(const GemvTask& t, const float* vperm, const float* vsum, const float* vsc) {
+    GemvRegs r;
+    gemv_load(t, r);   // every load of the task in flight before the arithmetic
+    return gemv_dot(t, r, vperm, vsum, vsc);
+}
+
+// Thread 0 asks L2 to fetch the down blocks of (expert list entry, m-tile) chunks
+// blockIdx.x, blockIdx.x + gridDim.x, ...: one m-tile's whole k range is one contiguous run.
+// experts == nullptr stands for the shared expert (group E).
+__device__ __forceinline__ void prefetch_down(const Ctx& c, const int* experts, int nexp) {
+    if (threadIdx.x != 0) return;
+    const int MTd = c.H / 128, KSd = c.I / 64;
+    for (int ch = blockIdx.x; ch < nexp * MTd; ch += gridDim.x) {
+        const int e = experts ? experts[ch / MTd] : c.E, mt = ch % MTd;
+        prefetch_l2(c.w_dn + ((size_t)e * MTd + mt) * KSd * kBlockBytes, (uint32_t)(KSd * kBlockBytes));
+    }
 }
 
 // Per-64-element group power-of-two scaling (see decode.cu): vperm in slot order, group sums, 2^(149-K).
@@ -179,11 +208,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
     float* rpart = c.dfz.rpart;      // [4][E]
     float* gu = c.dfz.gu;            // [slots][kGuKR][2I]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * kFWarps + warp;
+    const int gw = warp * gridDim.x + blockIdx.x;   // task t -> SM t % grid: a phase spreads over every SM
     const int NW = gridDim.x * kFWarps;
     const uint16_t* xr = c.x;        // T == 1
 
     // ------------------------------------------------------------------ phase 0
+    if (c.has_shared) prefetch_down(c, nullptr, 1);   // the shared expert's down blocks, needed in phase 2
     for (int i = threadIdx.x; i < H; i += kFThreads) x32[i] = __uint_as_float((uint32_t)xr[i] << 16);
     if (threadIdx.x == 0) *abort_flag = 0;
     __syncthreads();
@@ -280,6 +310,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
         if (blockIdx.x == 0 && lane == 0) c.sg[0] = selg[32];
     }
     __syncthreads();
+    prefetch_down(c, sel, k);   // the routed experts' down blocks stream into L2 during gate/up
     {
         const int n_tasks = k * MTg * 4 * kGuKR;
         for (int task = gw; task < n_tasks; task += NW) {
@@ -305,6 +336,17 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
         const int j = vb % nslot, bi = vb / nslot;
         const int e = (j < k) ? sel[j] : E;
         const float gate = (j < k) ? selg[j] : selg[32];
+        const int task = bi * kFWarps + warp;
+        GemvTask t;
+        GemvRegs wr;
+        if (task < tasks_per_slot) {   // weight loads first: they overlap the act staging below
+            const int mt = task / (4 * kDnKR), q = (task / kDnKR) & 3, kr = task % kDnKR;
+            t.blocks = c.w_dn + ((size_t)e * MTd + mt) * KSd * kBlockBytes;
+            t.row = 32 * q + lane;
+            t.k0 = kr * KSd / kDnKR;
+            t.k1 = (kr + 1) * KSd / kDnKR;
+            gemv_load(t, wr);
+        }
         __syncthreads();
         // act = silu(G) * U for this slot, from the k-range partials (gate row / up row of column i)
         stage_groups(I, [&](int i) {
@@ -319,15 +361,9 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
             return G * U / (1.f + expf(-G));
         }, aperm, asum, asc);
         __syncthreads();
-        const int task = bi * kFWarps + warp;
         if (task < tasks_per_slot) {
-            const int mt = task / (4 * kDnKR), q = (task / kDnKR) & 3, kr = task % kDnKR;
-            GemvTask t;
-            t.blocks = c.w_dn + ((size_t)e * MTd + mt) * KSd * kBlockBytes;
-            t.row = 32 * q + lane;
-            t.k0 = kr * KSd / kDnKR;
-            t.k1 = (kr + 1) * KSd / kDnKR;
-            const float y = run_gemv(t, aperm, asum, asc) * gate;
+            const int mt = task / (4 * kDnKR), q = (task / kDnKR) & 3;
+            const float y = gemv_dot(t, wr, aperm, asum, asc) * gate;
             const int h = mt * 128 + t.row;
             atomicAdd(&c.dfz.outacc[h], y);
             __threadfence();

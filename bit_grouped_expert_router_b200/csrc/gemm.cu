@@ -13,10 +13,12 @@
 // Shaped by measurement on this part: every TMA operation costs an SM at least ~360 cycles
 // whatever its size, while big copies stream at ~90 B/clk.  So the weight blocks travel four
 // k-steps per copy, the token tile is a single box per k-step whose height (64/128/256 rows)
-// follows the tile's token count, and the three operand rings are sized separately:
+// follows the tile's token count, and the three operand rings are sized separately (the token
+// ring's refill waits on L2, the A ring's only on the transform warps):
 //   weight ring  kWS stages x kWB blocks   (producer -> transform)
 //   token ring   kBS stages x 256 x 64     (producer -> MMA)
 //   A ring       kAS stages x 128 x 64     (transform -> MMA)
+// Barrier arrivals are one per warp.
 //
 //   gate/up kernel : per tile (expert, 128 interleaved gate/up rows, <=256 tokens), K = H.
 //                    B = the expert's bucketed fp16 token rows (the shared expert reads the fp16
@@ -57,10 +59,19 @@ constexpr int kAccCols = kBN;
 static_assert(2 * kAccCols <= kTmemCols, "TMEM budget");
 static_assert(kBN == 256, "token tile");
 
-constexpr int kWB = 4;   // weight blocks per bulk copy
+#ifndef GEMM_KWB
+#define GEMM_KWB 4
+#endif
+constexpr int kWB = GEMM_KWB;   // weight blocks per bulk copy
 constexpr int kWS = 2;   // weight ring stages
-constexpr int kBS = 3;   // token ring stages
-constexpr int kAS = 3;   // A ring stages
+#ifndef GEMM_KBS
+#define GEMM_KBS 3
+#endif
+#ifndef GEMM_KAS
+#define GEMM_KAS 3
+#endif
+constexpr int kBS = GEMM_KBS;   // token ring stages
+constexpr int kAS = GEMM_KAS;   // A ring stages
 
 constexpr int kATileBytes = 128 * 128;      // 128 weight rows x 64 fp16
 constexpr int kBTileBytes = kBN * 128;      // up to 256 token rows x 64 fp16
@@ -98,15 +109,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
     float** meta_row = reinterpret_cast<float**>(smem + kOffMeta);
     float* meta_gate = reinterpret_cast<float*>(smem + kOffMeta + 2 * kBN * 8);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* wfull = bars;                 // weight blocks landed      (1 arrive + tx)
-    uint64_t* wempty = wfull + kWS;         // weight blocks consumed    (256 arrives)
-    uint64_t* bfull = wempty + kWS;         // token tile landed         (1 arrive + tx)
-    uint64_t* bempty = bfull + kBS;         // token tile's MMAs done    (commit)
-    uint64_t* afull = bempty + kBS;         // fp16 A tile written       (256 arrives)
-    uint64_t* aempty = afull + kAS;         // A tile's MMAs done        (commit)
-    uint64_t* accfull = aempty + kAS;       // accumulator ready         (commit)
-    uint64_t* accempty = accfull + 2;       // accumulator drained       (256 arrives)
-    uint64_t* drainbar = accfull + 4;       // MMA drain on abort        (commit)
+    uint64_t* wfull = bars;                 // weight blocks landed          (1 arrive + tx)
+    uint64_t* wempty = wfull + kWS;         // weight blocks consumed        (1 arrive per transform warp)
+    uint64_t* bfull = wempty + kWS;         // token tile landed             (1 arrive + tx)
+    uint64_t* bempty = bfull + kBS;         // token tile's MMAs done        (commit)
+    uint64_t* afull = bempty + kBS;         // fp16 A tile written           (1 arrive per transform warp)
+    uint64_t* aempty = afull + kAS;         // A tile's MMAs done            (commit)
+    uint64_t* accfull = aempty + kAS;       // accumulator ready             (commit)
+    uint64_t* accempty = accfull + 2;       // accumulator drained           (1 arrive per epilogue warp)
+    uint64_t* drainbar = accfull + 4;       // MMA drain on abort            (commit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -118,19 +129,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kWS; ++s) {
             mbar_init(&wfull[s], 1);
-            mbar_init(&wempty[s], 32 * kTransformWarps);
+            mbar_init(&wempty[s], kTransformWarps);
         }
         for (int s = 0; s < kBS; ++s) {
             mbar_init(&bfull[s], 1);
             mbar_init(&bempty[s], 1);
         }
         for (int s = 0; s < kAS; ++s) {
-            mbar_init(&afull[s], 32 * kTransformWarps);
+            mbar_init(&afull[s], kTransformWarps);
             mbar_init(&aempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accfull[b], 1);
-            mbar_init(&accempty[b], 32 * kEpiWarps);
+            mbar_init(&accempty[b], kEpiWarps);
         }
         mbar_init(drainbar, 1);
         *abort_flag = 0;
@@ -260,8 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
             const int4 tile = c.tiles1[tau / MT];
             if (!tile_ok(tile, c)) continue;
             for (int kc = 0; kc < KS; ++kc) {
-                if (kc % kWB == 0 && !mbar_wait(&wfull[ws], wph, abort_flag, c.status)) goto transform_done;
-                if (!mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status)) goto transform_done;
+                // waits end the same way for the whole warp (the vote), so no lane is left behind
+                bool ok = kc % kWB != 0 || mbar_wait(&wfull[ws], wph, abort_flag, c.status);
+                ok = ok && mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status);
+                if (!__all_sync(0xffffffffu, ok)) goto transform_done;
                 const uint8_t* blk = wsm + ws * kWStageBytes + (kc % kWB) * kBlockBytes;
                 const uint4 cw = *reinterpret_cast<const uint4*>(blk + half * 2048 + row * 16);
                 const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
@@ -283,10 +296,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                     *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(r[0], r[1], r[2], r[3]);
                 }
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
-                mbar_arrive(&afull[as]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&afull[as]);
                 if (++as == kAS) { as = 0; aph ^= 1u; }
                 if (kc % kWB == kWB - 1 || kc == KS - 1) {   // this weight stage is used up
-                    mbar_arrive(&wempty[ws]);
+                    if (lane == 0) mbar_arrive(&wempty[ws]);
                     if (++ws == kWS) { ws = 0; wph ^= 1u; }
                 }
             }
@@ -314,7 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                 }
                 named_bar(1, 32 * kEpiWarps);
             }
-            if (!mbar_wait(&accfull[ab], aph, abort_flag, c.status)) goto epilogue_done;
+            {
+                const bool ok = mbar_wait(&accfull[ab], aph, abort_flag, c.status);
+                if (named_bar_or(2, 32 * kEpiWarps, !ok)) goto epilogue_done;   // the group leaves together
+            }
             tc_fence_after();
             const uint32_t taddr = tmem + lane_base + ab * kAccCols;
             if (GATEUP) {
@@ -337,7 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&accempty[ab]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[ab]);
                 named_bar(1, 32 * kEpiWarps);
                 const size_t I = (size_t)c.I;
                 for (int idx = etid; idx < nvalid * 8; idx += 32 * kEpiWarps) {
@@ -362,7 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&accempty[ab]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[ab]);
             }
         }
     epilogue_done:
