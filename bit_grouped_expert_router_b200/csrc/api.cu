@@ -137,7 +137,7 @@ Layout make_layout(const moe_config& c) {
     L.o_dfz_gu = take(sizeof(float) * (size_t)(L.k + 1) * 4 * 2 * L.I);
     L.o_dfz_outacc = take(sizeof(float) * (size_t)L.H);
     L.o_dfz_cnt = take(sizeof(unsigned) * (size_t)(L.H / 32));
-    L.o_dfz_bar = take(sizeof(unsigned) * 2);
+    L.o_dfz_bar = take(sizeof(unsigned long long) * 16 * 32);
     L.ws_bytes = o;
     return L;
 }
@@ -442,7 +442,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.dfz.gu = reinterpret_cast<float*>(ws + L.o_dfz_gu);
     c.dfz.outacc = reinterpret_cast<float*>(ws + L.o_dfz_outacc);
     c.dfz.cnt = reinterpret_cast<unsigned*>(ws + L.o_dfz_cnt);
-    c.dfz.bar = reinterpret_cast<unsigned*>(ws + L.o_dfz_bar);
+    c.dfz.bar = reinterpret_cast<unsigned long long*>(ws + L.o_dfz_bar);
 
     for (int hs = 0; hs < 3 && rc == MOE_OK; ++hs) {
         const int box = 64 << hs;   // token tile box: 64, 128 or 256 rows
@@ -550,7 +550,7 @@ int moe_status(moe_handle* h) {
     CUDA_TRY(cudaMemset(h->base.status, 0, sizeof s));
     if (s & MOE_STATUS_TIMEOUT) {
         // a kernel gave up part-way: put the fused decode's self-cleaning state back to zero
-        CUDA_TRY(cudaMemset(h->base.dfz.bar, 0, 2 * sizeof(unsigned)));
+        CUDA_TRY(cudaMemset(h->base.dfz.bar, 0, sizeof(unsigned long long) * 16 * 32));
         CUDA_TRY(cudaMemset(h->base.dfz.cnt, 0, sizeof(unsigned) * (size_t)(h->L.H / 32)));
         CUDA_TRY(cudaMemset(h->base.dfz.outacc, 0, sizeof(float) * (size_t)h->L.H));
         return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");

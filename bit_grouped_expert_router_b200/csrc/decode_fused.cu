@@ -22,7 +22,7 @@
 // at kernel start, the routed experts' right after top-k), and each phase-2 warp issues its
 // weight loads before it builds act, so phase 2 mostly waits on L2, not HBM.  GEMV arithmetic as
 // in decode.cu.
-// Grid barrier: arrival counter + generation word in the workspace; waits are bounded (1 s), on a
+// Grid barrier: ever-growing arrival counters in the workspace; waits are bounded (1 s), on a
 // timeout the status word records it and moe_status resets the barrier state.
 #include "common.cuh"
 #include "kernels.h"
@@ -75,22 +75,38 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// Sense-by-generation grid barrier: bar[0] arrivals, bar[1] generation.  Bounded.
-__device__ bool grid_barrier(unsigned* bar, unsigned nblocks, uint32_t* status, volatile int* abort_flag) {
+// Grid barrier on kBarCounters counters that only grow, 256 bytes apart: CTA b adds 1 (release,
+// GPU scope) to counter b mod kBarCounters, so few same-address atomics queue behind each other;
+// the barrier index follows from the value it found, and warp 0 then polls every counter (acquire)
+// until each has received one arrival per CTA mapped to it for this barrier.  No reset: between
+// barriers every counter holds a multiple of its CTA count (the handle zeroes them after a
+// timeout).  Bounded.
+constexpr int kBarCounters = 16;
+constexpr int kBarStride = 32;   // u64 words between counters
+
+__device__ bool grid_barrier(unsigned long long* ctr, unsigned nblocks, uint32_t* status, volatile int* abort_flag) {
     __syncthreads();
-    bool ok = true;
-    if (threadIdx.x == 0) {
-        volatile unsigned* gen = bar + 1;
-        const unsigned g = *gen;
-        __threadfence();
-        const unsigned arrived = atomicAdd(bar, 1u);
-        if (arrived == nblocks - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            atomicAdd(bar + 1, 1u);
-        } else {
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const unsigned nc = nblocks < (unsigned)kBarCounters ? nblocks : (unsigned)kBarCounters;
+        auto members = [&](unsigned j) { return nblocks / nc + (j < nblocks % nc ? 1u : 0u); };
+        unsigned long long b = 0;
+        if (lane == 0) {
+            const unsigned j = blockIdx.x % nc;
+            unsigned long long old;
+            asm volatile("atom.add.release.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr + (size_t)j * kBarStride) : "memory");
+            b = old / members(j);
+        }
+        b = __shfl_sync(0xffffffffu, b, 0);
+        bool ok = true;
+        if ((unsigned)lane < nc) {
+            const unsigned long long target = (b + 1) * members((unsigned)lane);
+            const unsigned long long* p = ctr + (size_t)lane * kBarStride;
             const unsigned long long t0 = globaltimer_ns();
-            while (*gen == g) {
+            while (true) {
+                unsigned long long v;
+                asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+                if (v >= target) break;
                 if (globaltimer_ns() - t0 > kWaitLimitNs) {
                     set_status(status, MOE_STATUS_TIMEOUT);
                     ok = false;
@@ -98,11 +114,18 @@ __device__ bool grid_barrier(unsigned* bar, unsigned nblocks, uint32_t* status, 
                 }
             }
         }
-        __threadfence();
-        *abort_flag = ok ? 0 : 1;
+        ok = __all_sync(0xffffffffu, ok);
+        if (lane == 0) *abort_flag = ok ? 0 : 1;
     }
     __syncthreads();
     return *abort_flag == 0;
+}
+
+// Order-preserving map of a float to an unsigned key (-0 first made +0, so equal floats give
+// equal keys).
+__device__ __forceinline__ uint32_t ord_key(float v) {
+    const uint32_t u = __float_as_uint(v + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 struct GemvTask {  // one warp: 32 rows (lane = row) of one m-tile, k-steps [k0, k1)
@@ -153,11 +176,12 @@ __device__ __forceinline__ float run_gemv(const GemvTask& t, const float* vperm,
     return gemv_dot(t, r, vperm, vsum, vsc);
 }
 
-// Thread 0 asks L2 to fetch the down blocks of (expert list entry, m-tile) chunks
+// One thread asks L2 to fetch the down blocks of (expert list entry, m-tile) chunks
 // blockIdx.x, blockIdx.x + gridDim.x, ...: one m-tile's whole k range is one contiguous run.
-// experts == nullptr stands for the shared expert (group E).
+// experts == nullptr stands for the shared expert (group E).  Not thread 0: its grid-barrier
+// release would wait for the prefetches to finish.
 __device__ __forceinline__ void prefetch_down(const Ctx& c, const int* experts, int nexp) {
-    if (threadIdx.x != 0) return;
+    if (threadIdx.x != 32) return;
     const int MTd = c.H / 128, KSd = c.I / 64;
     for (int ch = blockIdx.x; ch < nexp * MTd; ch += gridDim.x) {
         const int e = experts ? experts[ch / MTd] : c.E, mt = ch % MTd;
@@ -214,6 +238,22 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
 
     // ------------------------------------------------------------------ phase 0
     if (c.has_shared) prefetch_down(c, nullptr, 1);   // the shared expert's down blocks, needed in phase 2
+    const int n_router = E * 4;
+    const int n_shared = c.has_shared ? MTg * 4 * kGuKR : 0;
+    const int hq = H / 4;   // router quarter row
+    // A warp's first task reads weights that do not depend on x: they are requested into L2 before
+    // x is staged, so the two memory latencies overlap (bulk L2 prefetch, lane 0 of the warp).
+    if (lane == 0) {
+        if (gw < n_router) {
+            prefetch_l2(c.router32 + (size_t)(gw >> 2) * H + (gw & 3) * hq, (uint32_t)(hq * sizeof(float)));
+        } else if (gw < n_router + n_shared) {
+            const int s0 = gw - n_router;
+            const int mt = s0 / (4 * kGuKR), q = (s0 / kGuKR) & 3, kr = s0 % kGuKR;
+            const int k0 = kr * KSg / kGuKR, k1 = (kr + 1) * KSg / kGuKR;
+            if (q == 0 && k1 > k0)   // the four row quarters share these blocks
+                prefetch_l2(c.w_gu + (((size_t)E * MTg + mt) * KSg + k0) * kBlockBytes, (uint32_t)((k1 - k0) * kBlockBytes));
+        }
+    }
     for (int i = threadIdx.x; i < H; i += kFThreads) x32[i] = __uint_as_float((uint32_t)xr[i] << 16);
     if (threadIdx.x == 0) *abort_flag = 0;
     __syncthreads();
@@ -229,34 +269,29 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
         for (int w = 0; w < kFWarps; ++w) z += red[w];
         selg[32] = c.has_shared ? 1.f / (1.f + expf(-z)) : 0.f;
     }
-    {
-        const int n_router = E * 4;
-        const int n_shared = c.has_shared ? MTg * 4 * kGuKR : 0;
-        for (int task = gw; task < n_router + n_shared; task += NW) {
-            if (task < n_router) {
-                const int e = task >> 2, kq = task & 3;
-                const int hq = H / 4;
-                const float* wrow = c.router32 + (size_t)e * H + kq * hq;
-                float d = 0.f;
+    for (int task = gw; task < n_router + n_shared; task += NW) {
+        if (task < n_router) {
+            const int e = task >> 2, kq = task & 3;
+            const float* wrow = c.router32 + (size_t)e * H + kq * hq;
+            float d = 0.f;
 #pragma unroll 4
-                for (int h = lane * 4; h < hq; h += 128) {
-                    const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + h));
-                    const float4 xv = *reinterpret_cast<const float4*>(x32 + kq * hq + h);
-                    d = fmaf(wv.x, xv.x, fmaf(wv.y, xv.y, fmaf(wv.z, xv.z, fmaf(wv.w, xv.w, d))));
-                }
-                d = warp_sum(d);
-                if (lane == 0) rpart[kq * E + e] = d;
-            } else {
-                const int s = task - n_router;
-                const int mt = s / (4 * kGuKR), q = (s / kGuKR) & 3, kr = s % kGuKR;
-                GemvTask t;
-                t.blocks = c.w_gu + ((size_t)E * MTg + mt) * KSg * kBlockBytes;   // shared expert = group E
-                t.row = 32 * q + lane;
-                t.k0 = kr * KSg / kGuKR;
-                t.k1 = (kr + 1) * KSg / kGuKR;
-                const float v = run_gemv(t, xperm, xsum, xsc);
-                gu[((size_t)k * kGuKR + kr) * (2 * I) + mt * 128 + t.row] = v;
+            for (int h = lane * 4; h < hq; h += 128) {
+                const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + h));
+                const float4 xv = *reinterpret_cast<const float4*>(x32 + kq * hq + h);
+                d = fmaf(wv.x, xv.x, fmaf(wv.y, xv.y, fmaf(wv.z, xv.z, fmaf(wv.w, xv.w, d))));
             }
+            d = warp_sum(d);
+            if (lane == 0) rpart[kq * E + e] = d;
+        } else {
+            const int s = task - n_router;
+            const int mt = s / (4 * kGuKR), q = (s / kGuKR) & 3, kr = s % kGuKR;
+            GemvTask t;
+            t.blocks = c.w_gu + ((size_t)E * MTg + mt) * KSg * kBlockBytes;   // shared expert = group E
+            t.row = 32 * q + lane;
+            t.k0 = kr * KSg / kGuKR;
+            t.k1 = (kr + 1) * KSg / kGuKR;
+            const float v = run_gemv(t, xperm, xsum, xsc);
+            gu[((size_t)k * kGuKR + kr) * (2 * I) + mt * 128 + t.row] = v;
         }
     }
     if (!grid_barrier(c.dfz.bar, gridDim.x, c.status, abort_flag)) return;
@@ -272,28 +307,26 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
     }
     __syncthreads();
     if (warp == 0) {
-        float l[8];
+        // top-k by logit, ties to the lower expert index: per round one warp-wide max of the keys
+        // and one min of the indices holding it (two redux instructions)
+        uint32_t key[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) l[i] = logits[lane + 32 * i];
+        for (int i = 0; i < 8; ++i) key[i] = ord_key(logits[lane + 32 * i]);
         unsigned taken = 0;
         int my_e = 0;
         float my_v = 0.f;
         for (int j = 0; j < k; ++j) {
-            float bv = 0.f;
-            int be = 0x7fffffff;
+            uint32_t best = 0;
+            int bi = -1;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || l[i] > bv)) { bv = l[i]; be = e; }
+                if (lane + 32 * i < E && !((taken >> i) & 1u) && (bi < 0 || key[i] > best)) { best = key[i]; bi = i; }
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            if (lane == j) { my_e = be; my_v = bv; }
+            const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+            const uint32_t cand = (bi >= 0 && best == m) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
+            const uint32_t be = __reduce_min_sync(0xffffffffu, cand);
+            if ((int)(be & 31u) == lane) taken |= 1u << (be >> 5);
+            if (lane == j) { my_e = (int)be; my_v = logits[be & 255u]; }
         }
         const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
         const float p = lane < k ? expf(my_v - vmax) : 0.f;
@@ -366,13 +399,17 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
             const float y = gemv_dot(t, wr, aperm, asum, asc) * gate;
             const int h = mt * 128 + t.row;
             atomicAdd(&c.dfz.outacc[h], y);
-            __threadfence();
             __syncwarp();
             unsigned last = 0;
-            if (lane == 0) last = (atomicAdd(&c.dfz.cnt[mt * 4 + q], 1u) == (unsigned)expected - 1) ? 1u : 0u;
+            if (lane == 0) {
+                // acq_rel: releases this warp's additions, and the last arriver acquires everyone's
+                unsigned old;
+                asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(&c.dfz.cnt[mt * 4 + q]) : "memory");
+                last = old == (unsigned)expected - 1 ? 1u : 0u;
+            }
             last = __shfl_sync(0xffffffffu, last, 0);
+            __syncwarp();
             if (last) {
-                __threadfence();
                 const float v = atomicExch(&c.dfz.outacc[h], 0.f);
                 c.out[h] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
                 if (lane == 0) atomicExch(&c.dfz.cnt[mt * 4 + q], 0u);

@@ -32,13 +32,14 @@ struct RepackArgs {
 };
 
 // Workspace of the fused batch-1 decode kernel.  outacc and cnt are zero between calls (the
-// kernel re-zeroes what it used); bar is the grid barrier {arrivals, generation}.
+// kernel re-zeroes what it used); bar holds grid-barrier arrival counts (between calls each a
+// multiple of the number of CTAs that arrive on it).
 struct DecodeFusedWs {
     float* rpart;    // [4][E] quarter-row router partial logits
     float* gu;       // [k+1][4][2I] gate/up k-range partial sums
     float* outacc;   // [H] fp32 output accumulator
     unsigned* cnt;   // [H/32] arrivals per 32-row output chunk
-    unsigned* bar;   // [2]
+    unsigned long long* bar;   // [16 x 32] grid-barrier arrival counters (256 B apart), only ever incremented
 };
 
 // Everything a forward-path kernel needs (passed by value).
