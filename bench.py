@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -252,7 +253,7 @@ def run_prefill(args, dist, peaks, peak_src):
         a = f_gu / (prof["gemm_gateup"]["avg_us"] * 1e-6) / 1e12
         roof = {"bound": "tensor", "kernel": "gemm_gateup (tcgen05 grouped GEMM + SwiGLU)",
                 "achieved": round(a, 1), "peak": peak_tf, "unit": "TFLOP/s", "frac": round(a / peak_tf, 4),
-                "traffic": None, "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16 dense rate)",
+                "traffic": profiled_traffic("gemm_gateup"), "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16 dense rate)",
                 "flops_per_launch": f_gu}
     gg = None
     if "gemm_gateup" in prof and "gemm_down" in prof:
@@ -343,20 +344,38 @@ def run_decode(args, dist, peaks, peak_src):
             "gpu_launches_per_step": (1 if "decode_fused" in prof else 4) * n_layers}
 
 
+# ------------------------------------------------------------------------------------ ncu traffic
+def profiled_traffic(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary, or None when
+    the kernel sources changed since that capture (the summary records their sha256)."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    prof = os.path.join(here, "profiles", "grouped_gemm_prefill16k_zipf_1layer.md")
+    if not os.path.exists(prof):
+        return None
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(here, "bit_grouped_expert_router_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    text = open(prof).read()
+    m = re.search(r"kernel_sources_sha256_16: ([0-9a-f]{16})", text)
+    t = re.search(r"traffic_bytes_per_launch %s: (\d+)" % re.escape(kernel), text)
+    if not m or not t or m.group(1) != h.hexdigest()[:16]:
+        return None
+    return int(t.group(1))
+
+
 # ------------------------------------------------------------------------------------ CPU oracle
 def cpu_baseline(host0, x0, shape, target_s):
     import oracle
     ol = oracle.OracleLayer.from_shape(host0, shape)
-    n = 8
-    t0 = time.perf_counter()
-    ol.forward(x0, tokens=list(range(n)))
-    dt = time.perf_counter() - t0
-    n2 = int(min(shape.T - n, max(8, (target_s - dt) / max(dt / n, 1e-6))))
-    t1 = time.perf_counter()
-    if n2 > 0:
-        ol.forward(x0, tokens=list(range(n, n + n2)))
-    dt2 = time.perf_counter() - t1
-    total_n, total_t = (n + n2, dt + dt2)
+    # batches of 32 tokens until the target time is spent (or the chunk is used up)
+    total_n, t0 = 0, time.perf_counter()
+    while total_n < shape.T and time.perf_counter() - t0 < target_s:
+        b = min(32, shape.T - total_n)
+        ol.forward(x0, tokens=list(range(total_n, total_n + b)))
+        total_n += b
+    total_t = time.perf_counter() - t0
     return {"value": round(total_n / total_t, 3), "unit": "tokens/s", "cores": oracle.max_threads(),
             "kind": "oracle",
             "sample": f"{total_n} tokens of layer 0, chunk 0 through one MoE layer (fp64 oracle, "

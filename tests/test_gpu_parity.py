@@ -256,3 +256,25 @@ def test_decode_fused_and_unfused_agree_and_replay_in_a_graph():
         assert f.status() == M.MOE_OK
         f.close()
         u.close()
+
+
+# ---------------------------------------------------------------------------------------------
+# failure detection without a GPU fault
+def test_stalled_wait_times_out_and_the_context_stays_usable():
+    """A bounded device-side wait that runs out.  With the test-only stall flag the prefill
+    producer withholds every load, so the grouped GEMMs' consumer waits reach their limit: the
+    kernels unwind and return, the status word reads MOE_ERR_DEVICE_TIMEOUT, and afterwards a
+    normal layer on the same device computes correct results (the context was never lost)."""
+    shape = TINY
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    stalled = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=0, flags=M.MOE_FLAG_TEST_STALL)
+    stalled.forward(x.cuda())
+    torch.cuda.synchronize()
+    assert stalled.status() == M.MOE_ERR_DEVICE_TIMEOUT
+    assert stalled.status() == M.MOE_OK   # reading the status clears it
+    stalled.close()
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=0)
+    _forward_check(layer, ol, x)
+    layer.close()
