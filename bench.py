@@ -58,6 +58,7 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the prefill512 / prefill4k_zipf fractions")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle sample time")
     return ap.parse_args()
 
@@ -289,6 +290,89 @@ def run_prefill(args, dist, peaks, peak_src):
     return res
 
 
+def decode_gemv_only(shape, xs, reps, hbm, peak_src):
+    """The expert GEMV kernels alone: batch-1 decode through the multi-kernel chain (router, top-k,
+    gate/up GEMV, down GEMV) on 8 distinct layers; bytes = the k+1 experts' packed weights."""
+    import torch
+    from bit_grouped_expert_router_b200 import _lib as M
+    from bit_grouped_expert_router_b200 import synth
+    n = min(8, len(xs))
+    layers = []
+    for l in range(n):
+        w = synth.make_layer(shape, l, device="cuda")
+        layers.append(M.Layer.from_shape(w, shape, max_tokens=16, decode_max_tokens=16,
+                                         flags=M.MOE_FLAG_DECODE_UNFUSED))
+        del w
+    outs = [torch.empty((1, shape.H), dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+
+    def step():
+        for l in range(n):
+            layers[l].forward(xs[l], out=outs[l])
+
+    for _ in range(3):
+        step()
+    prof = profile_pass(layers, step, reps)
+    for L in layers:
+        assert L.status() == 0
+        L.close()
+    nexp = shape.k + 1
+    b = nexp * ((shape.I // 64) * (shape.H // 64) + (shape.H // 128) * (shape.I // 64)) * 4608
+    t = (prof["gemv_gateup"]["avg_us"] + prof["gemv_down"]["avg_us"]) * 1e-6
+    a = b / t / 1e9
+    return {"kernels": "gemv_gateup + gemv_down (unfused chain, eager, profiled)",
+            "us": round(t * 1e6, 3), "bytes": b, "achieved": round(a, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(a / hbm, 4), "peak_source": f"{peak_src} hbm_gbs",
+            "chain_kernels_us": {k: round(v["avg_us"], 2) for k, v in prof.items()}}
+
+
+def run_configs(args, dist, peaks, peak_src):
+    """The other prefill configurations' roofline fractions: prefill512 (HBM-bound: algorithmic
+    bytes = weights of the experts that receive a token + router + shared gate + x/out, over the
+    whole-layer time) and prefill4k_zipf (tensor-bound: MoE FLOPs over the two GEMMs' time), each
+    on 4 distinct layers (1.8 GB of weights, well above L2)."""
+    import torch
+    from bit_grouped_expert_router_b200 import synth
+    out = {}
+    expert_bytes = None
+    for name in ("prefill512", "prefill4k_zipf"):
+        shape = synth.WORKLOADS[name]
+        n = 4
+        layers, _ = build_stack(shape, n, shape.T, 16)
+        xs = [synth.make_x(shape, l, 0, device="cuda") for l in range(n)]
+        expert_bytes = (shape.I // 64) * (shape.H // 64) * 4608 + (shape.H // 128) * (shape.I // 64) * 4608
+
+        def step():
+            for l in range(n):
+                layers[l].forward(xs[l])
+
+        reps = max(args.steps, 5)
+        ms = timed(step, reps, 3, dist) / n
+        prof = profile_pass(layers, step, reps)
+        active = []
+        for l in range(n):
+            idx = layers[l].route(xs[l])["idx"]
+            active.append(int(torch.unique(idx).numel()) + (1 if shape.has_shared else 0))
+        for L in layers:
+            assert L.status() == 0
+            L.close()
+        f_gu, f_dn = gemm_flops(shape)
+        t_gemm = (prof["gemm_gateup"]["avg_us"] + prof["gemm_down"]["avg_us"]) * 1e-6
+        bytes_alg = statistics.mean(active) * expert_bytes + shape.E * shape.H * 4 + shape.H * 4 + 2 * shape.T * shape.H * 2
+        hbm, tf = peaks["hbm_gbs"], peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+        out[name] = {"tokens": shape.T, "layer_us": round(ms * 1000, 2),
+                     "layer_tokens_per_s": round(shape.T / (ms / 1000), 1),
+                     "active_experts_mean": statistics.mean(active),
+                     "hbm_frac_whole_layer": round(bytes_alg / (ms / 1000) / 1e9 / hbm, 4),
+                     "algorithmic_bytes": int(bytes_alg),
+                     "gemm_tflops": round((f_gu + f_dn) / t_gemm / 1e12, 1),
+                     "gemm_tensor_frac": round((f_gu + f_dn) / t_gemm / 1e12 / tf, 4),
+                     "kernels_us": {k: round(v["avg_us"], 1) for k, v in prof.items()},
+                     "peaks": f"{peak_src}: hbm_gbs {hbm}, bf16 sustained {tf} TFLOP/s"}
+        del xs
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_decode(args, dist, peaks, peak_src):
     import torch
     from bit_grouped_expert_router_b200 import synth
@@ -337,10 +421,12 @@ def run_decode(args, dist, peaks, peak_src):
         assert L.status() == 0
         L.close()
     del g
+    gemv_only = decode_gemv_only(shape, xs, max(args.steps, 20), hbm, peak_src)
     return {"metric": "MoE-layer decode us/token/layer (batch 1, 40 distinct layers, one CUDA graph)",
             "value": round(us_layer, 3), "unit": "us/token/layer", "higher_is_better": False,
             "whole_layer_hbm_frac": round(layer_bytes / (us_layer * 1e-6) / 1e9 / hbm, 4),
             "whole_layer_bytes": layer_bytes, "roofline": roof, "kernels": prof,
+            "gemv_kernels_only": gemv_only,
             "gpu_launches_per_step": (1 if "decode_fused" in prof else 4) * n_layers}
 
 
@@ -454,6 +540,8 @@ def main():
         if not args.no_decode:
             d = run_decode(args, dist, peaks, peak_src)
             line["decode"] = d
+        if not args.no_configs and dist.world == 1:
+            line["other_configs"] = run_configs(args, dist, peaks, peak_src)
         line["config"] = {"workload": args.workload, "tokens": shape.T * shape.chunks, "chunk": shape.T,
                           "layers": r["n_layers"], "H": shape.H, "I": shape.I, "E": shape.E, "k": shape.k,
                           "shared_expert": shape.has_shared, "zipf_s": shape.zipf_s,
