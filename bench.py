@@ -422,7 +422,7 @@ def run_decode(args, dist, peaks, peak_src):
         L.close()
     del g
     gemv_only = decode_gemv_only(shape, xs, max(args.steps, 20), hbm, peak_src)
-    return {"metric": "MoE-layer decode us/token/layer (batch 1, 40 distinct layers, one CUDA graph)",
+    return {"metric": DECODE_METRIC,
             "value": round(us_layer, 3), "unit": "us/token/layer", "higher_is_better": False,
             "whole_layer_hbm_frac": round(layer_bytes / (us_layer * 1e-6) / 1e9 / hbm, 4),
             "whole_layer_bytes": layer_bytes, "roofline": roof, "kernels": prof,
@@ -468,6 +468,23 @@ def cpu_baseline(host0, x0, shape, target_s):
                       f"{total_t:.1f} s); per-layer tokens/s comparable to value"}
 
 
+def prefill_metric(shape, n_layers):
+    return (f"MoE-layer prefill tokens/s ({shape.T * shape.chunks}-token prompt in {shape.T}-token chunks, "
+            f"{n_layers} layers; also decode us/token/layer)")
+
+
+DECODE_METRIC = "MoE-layer decode us/token/layer (batch 1, 40 distinct layers, one CUDA graph)"
+
+
+def prefill_config(args, shape, n_layers):
+    return {"workload": args.workload, "tokens": shape.T * shape.chunks, "chunk": shape.T,
+            "layers": n_layers, "H": shape.H, "I": shape.I, "E": shape.E, "k": shape.k,
+            "shared_expert": shape.has_shared, "zipf_s": shape.zipf_s,
+            "weights": "int4 g64 asymmetric, bf16 scale/bias (repacked fp16)",
+            "l2": "inputs larger than L2: 457 MB of weights per layer, 40 distinct layers",
+            "decode_workload": "decode (T=1, 40 layers, CUDA graph)"}
+
+
 def run_reference(args, dist):
     """The oracle as the reference arm: rank 0 only, bounded token sample per step."""
     if dist.rank != 0:
@@ -489,17 +506,20 @@ def run_reference(args, dist):
         if i >= args.warmup:
             t_tok.append(dt)
     ms = 1000.0 * sum(t_tok) / len(t_tok)
+    n_layers = args.layers or shape.layers
     if args.workload == "decode":
-        value, unit, hib, metric = ms * 1000.0 / per_step, "us/token/layer", False, \
-            "MoE-layer decode us/token/layer"
+        value, unit, hib, metric = ms * 1000.0 / per_step, "us/token/layer", False, DECODE_METRIC
+        config = {"workload": "decode", "T": 1, "H": shape.H, "I": shape.I, "E": shape.E, "k": shape.k,
+                  "layers": n_layers}
     else:
-        value, unit, hib, metric = per_step / (ms / 1000.0), "tokens/s", True, "MoE-layer prefill tokens/s"
+        # per-layer tokens/s: the same unit as the GPU arm's layer-tokens/s
+        value, unit, hib, metric = per_step / (ms / 1000.0), "tokens/s", True, prefill_metric(shape, n_layers)
+        config = prefill_config(args, shape, n_layers)
     sample = f"{per_step} tokens of layer 0 per step through one MoE layer (fp64 CPU oracle)"
     line = {"impl": "reference", "metric": metric, "value": round(value, 4), "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": hib,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "T": shape.T, "H": shape.H, "E": shape.E, "k": shape.k,
-                       "I": shape.I, "layers_sampled": 1},
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded random-init weights and activations)",
+            "config": config,
             "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": oracle.max_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -523,13 +543,12 @@ def main():
     line = None
     if args.workload == "decode":
         d = run_decode(args, dist, peaks, peak_src)
-        line = {"metric": d["metric"], "value": d["value"] / dist.world, "unit": d["unit"],
+        line = {"metric": DECODE_METRIC, "value": d["value"] / dist.world, "unit": d["unit"],
                 "higher_is_better": False, "roofline": d["roofline"], "decode_detail": d}
     else:
         r = run_prefill(args, dist, peaks, peak_src)
         shape = r["shape"]
-        line = {"metric": f"MoE-layer prefill tokens/s ({shape.T * shape.chunks}-token prompt in "
-                          f"{shape.T}-token chunks, {r['n_layers']} layers; also decode us/token/layer)",
+        line = {"metric": prefill_metric(shape, r["n_layers"]),
                 "value": round(r["value"], 1), "unit": "tokens/s", "higher_is_better": True,
                 "ms_per_step": round(r["ms"], 3), "roofline": r["roofline"], "grouped_gemm": r["grouped_gemm"],
                 "kernels": r["kernels"], "gpu_launches": r["launches"], "clocks": r["clocks"]}
@@ -542,12 +561,7 @@ def main():
             line["decode"] = d
         if not args.no_configs and dist.world == 1:
             line["other_configs"] = run_configs(args, dist, peaks, peak_src)
-        line["config"] = {"workload": args.workload, "tokens": shape.T * shape.chunks, "chunk": shape.T,
-                          "layers": r["n_layers"], "H": shape.H, "I": shape.I, "E": shape.E, "k": shape.k,
-                          "shared_expert": shape.has_shared, "zipf_s": shape.zipf_s,
-                          "weights": "int4 g64 asymmetric, bf16 scale/bias (repacked fp16)",
-                          "l2": "inputs larger than L2: 457 MB of weights per layer, 40 distinct layers",
-                          "decode_workload": "decode (T=1, 40 layers, CUDA graph)"}
+        line["config"] = prefill_config(args, shape, r["n_layers"])
     base = {"n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16", "data": "synthetic (seeded random-init weights and activations)"}
     for k, v in base.items():
