@@ -75,6 +75,40 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Dot of one weight row (lane = row of the blocks at wb) over k-steps [c0, c1) with activations in
+// slot order: every load of a chunk of up to D k-steps is issued before its arithmetic, so a warp
+// keeps D x 36 bytes per lane in flight instead of waiting out one memory latency per k-step.
+template <int D>
+__device__ __forceinline__ float row_dot(const uint8_t* wb, int row, int c0, int c1, const float* vperm,
+                                         const float* vsc, const float* vsum) {
+    float acc = 0.f;
+    for (int base = c0; base < c1; base += D) {
+        const int n = min(D, c1 - base);
+        uint4 v0[D], v1[D];
+        uint32_t sb[D];
+#pragma unroll
+        for (int i = 0; i < D; ++i) {
+            if (i < n) {
+                const uint8_t* blk = wb + (size_t)(base + i) * kBlockBytes;
+                v0[i] = __ldg(reinterpret_cast<const uint4*>(blk + row * 16));
+                v1[i] = __ldg(reinterpret_cast<const uint4*>(blk + 2048 + row * 16));
+                sb[i] = __ldg(reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < D; ++i) {
+            if (i < n) {
+                const int cc = base + i;
+                const float s = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
+                const float b = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
+                const float P = dot_group(v0[i], v1[i], vperm + 64 * cc);
+                acc += s * (P * vsc[cc]) + b * vsum[cc];
+            }
+        }
+    }
+    return acc;
+}
+
 constexpr int kGateupThreads = 512;
 
 __global__ void __launch_bounds__(kGateupThreads) gemv_gateup_kernel(Ctx c) {
@@ -119,18 +153,7 @@ __global__ void __launch_bounds__(kGateupThreads) gemv_gateup_kernel(Ctx c) {
     const int row = 32 * q + lane;
     const int c0 = ksp * KS / 4, c1 = (ksp + 1) * KS / 4;
     const uint8_t* wb = c.w_gu + ((size_t)g * MT + mt) * KS * kBlockBytes;
-    float acc = 0.f;
-    for (int cc = c0; cc < c1; ++cc) {
-        const uint8_t* blk = wb + (size_t)cc * kBlockBytes;
-        const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(blk + row * 16));
-        const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(blk + 2048 + row * 16));
-        const uint32_t sb = __ldg(reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4));
-        const float s = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
-        const float b = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
-        const float P = dot_group(v0, v1, xperm + 64 * cc);
-        acc += s * (P * xsc[cc]) + b * xsum[cc];
-    }
-    red[ksp * 128 + row] = acc;
+    red[ksp * 128 + row] = row_dot<8>(wb, row, c0, c1, xperm, xsc, xsum);
     __syncthreads();
 
     // ---- SwiGLU on the 64 columns of this m-tile, scaled for the down GEMV
@@ -165,7 +188,7 @@ __global__ void __launch_bounds__(kGateupThreads) gemv_gateup_kernel(Ctx c) {
         c.dscale[(size_t)c.T * (c.k + 1) * MT + ((size_t)t * (c.k + 1) + j) * MT + mt] = red[0] + red[1] + red[2] + red[3];
 }
 
-__global__ void gemv_down_kernel(Ctx c) {
+__global__ void __launch_bounds__(1024) gemv_down_kernel(Ctx c) {
     extern __shared__ __align__(16) float sm[];
     const int hc = blockIdx.x, t = blockIdx.y;
     const int nslot = c.k + c.has_shared;
@@ -191,18 +214,7 @@ __global__ void gemv_down_kernel(Ctx c) {
             const float* sums = c.dscale + (size_t)c.T * (c.k + 1) * KS + ((size_t)t * (c.k + 1) + j) * KS;
             const uint8_t* wb = c.w_dn + ((size_t)g * MT + mt) * KS * kBlockBytes;
             const int c0 = ksp * KS / 2, c1 = (ksp + 1) * KS / 2;
-            float acc = 0.f;
-            for (int cc = c0; cc < c1; ++cc) {
-                const uint8_t* blk = wb + (size_t)cc * kBlockBytes;
-                const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(blk + row * 16));
-                const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(blk + 2048 + row * 16));
-                const uint32_t sb = __ldg(reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4));
-                const float s = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
-                const float b = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
-                const float P = dot_group(v0, v1, aperm + j * c.I + 64 * cc);
-                acc += s * (P * sc[cc]) + b * sums[cc];
-            }
-            contrib = acc * gate;
+            contrib = row_dot<4>(wb, row, c0, c1, aperm + j * c.I, sc, sums) * gate;
         } else if (lane == 0) {
             set_status(c.status, MOE_STATUS_BOUNDS);
         }
@@ -229,6 +241,7 @@ cudaError_t launch_gemv_gateup(const Ctx& c, cudaStream_t st) {
 cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st) {
     const int nslot = c.k + c.has_shared;
     const int threads = 64 * nslot;
+    if (threads > 1024) return cudaErrorInvalidConfiguration;   // k + shared > 16 slots
     const size_t smem = sizeof(float) * ((size_t)nslot * c.I + (size_t)threads);
     dim3 grid(c.H / 32, c.T);
     gemv_down_kernel<<<grid, threads, smem, st>>>(c);

@@ -89,7 +89,9 @@ typedef struct {
     int32_t has_shared;        /* 1: one always-on shared expert with a sigmoid gate */
     int32_t max_tokens;        /* largest T that moe_forward / moe_route accept */
     int32_t decode_max_tokens; /* T <= this runs the sparse-GEMV decode path; larger T runs the
-                                  bucketed grouped-GEMM prefill path.  0 = always prefill path. */
+                                  bucketed grouped-GEMM prefill path.  0 = always prefill path.
+                                  With decode_max_tokens >= 2 (or MOE_FLAG_DECODE_UNFUSED) the
+                                  multi-kernel GEMV path needs top_k + has_shared <= 16. */
     uint32_t flags;            /* MOE_FLAG_* */
 } moe_config;
 
