@@ -146,6 +146,20 @@ def test_full_prefill_workloads(name, layer_idx, chunk):
     layer.close()
 
 
+def test_one_16k_token_call_at_the_largest_sizes():
+    """All 16384 tokens of a prompt in one call (max_tokens = 16384): the largest buckets (the
+    skewed routing sends ~16k rows to its hottest expert), the longest tile list and the biggest
+    workspace.  Routing and bucketing checked for every token, outputs on 256 sampled tokens."""
+    shape = synth.shape_with(synth.WORKLOADS["prefill16k_zipf"], T=16384)
+    w = synth.make_layer(shape, 0)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol, 0, 0)
+    layer = _layer(w, shape, max_tokens=16384, decode_max_tokens=16)
+    _route_check(layer, ol, x, shape)
+    print("16k in one call", _forward_check(layer, ol, x, tokens=_sample(shape.T, 256, 11)))
+    layer.close()
+
+
 @pytest.mark.parametrize("layer_idx", [0, 39])
 def test_full_decode_workload(layer_idx):
     shape, w, ol, x = _full("decode", layer_idx, 0, T=16)
