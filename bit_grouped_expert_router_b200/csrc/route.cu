@@ -94,44 +94,79 @@ __device__ __forceinline__ uint32_t bf16x2_to_half2_bits(uint32_t w, bool* range
 // Shared gate: sigmoid(x . w_sg).  Prefill path (do_hist): count the token's experts into the
 // histogram row of its 64-token bucketing block (global atomics; the scatter kernel re-zeroes the
 // row after use) and zero the token's fp32 accumulator row for the down-projection combine.
+// Order-preserving map of a float to an unsigned key (-0 first made +0, so equal floats give
+// equal keys).
+__device__ __forceinline__ uint32_t ord_key(float v) {
+    const uint32_t u = __float_as_uint(v + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
     const int lane = lane_id();
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= c.T) return;
+    // logits: the partial sums of expert e = lane + 32 i, summed in split order, plus the bias
     float l[8];
+    if (c.ks == 4) {   // the tensor-core router's four partial sums: every load issued first
+        float pq[4][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        float v = -INFINITY;
-        if (e < c.E) {
-            float s = 0.f;
-            for (int q = 0; q < c.ks; ++q) s += c.part[((size_t)q * c.T + t) * c.E + e];
-            s += c.rbias[e];
-            v = (s != s) ? -INFINITY : s;
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane + 32 * i;
+                pq[q][i] = e < c.E ? c.part[((size_t)q * c.T + t) * c.E + e] : 0.f;
+            }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            const float s = (((pq[0][i] + pq[1][i]) + pq[2][i]) + pq[3][i]) + (e < c.E ? c.rbias[e] : 0.f);
+            l[i] = (e < c.E && s == s) ? s : -INFINITY;
         }
-        l[i] = v;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            float v = -INFINITY;
+            if (e < c.E) {
+                float s = 0.f;
+                for (int q = 0; q < c.ks; ++q) s += c.part[((size_t)q * c.T + t) * c.E + e];
+                s += c.rbias[e];
+                v = (s != s) ? -INFINITY : s;
+            }
+            l[i] = v;
+        }
     }
+    // top k by logit, ties to the lower expert index: per pick one warp-wide max of the keys and
+    // one min of the indices holding it
+    uint32_t key[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) key[i] = ord_key(l[i]);
     unsigned taken = 0;
     int my_e = 0;
     float my_v = 0.f;
     for (int j = 0; j < c.k; ++j) {
-        float bv = 0.f;
-        int be = 0x7fffffff;
+        uint32_t best = 0;
+        int bi = -1;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int e = lane + 32 * i;
-            if (e < c.E && !((taken >> i) & 1u)) {
-                if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
-            }
+            if (lane + 32 * i < c.E && !((taken >> i) & 1u) && (bi < 0 || key[i] > best)) { best = key[i]; bi = i; }
         }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = (bi >= 0 && best == m) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
+        const uint32_t be = __reduce_min_sync(0xffffffffu, cand);
+        if ((int)(be & 31u) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) my_e = (int)be;
+    }
+    // each lane j < k fetches the value of its pick from the lane that holds it
+    {
+        const int src = my_e & 31, slot = my_e >> 5;
+        float v = 0.f;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+        for (int i = 0; i < 8; ++i) {
+            const float cand = __shfl_sync(0xffffffffu, l[i], src);
+            if (i == slot) v = cand;
         }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        if (lane == j) { my_e = be; my_v = bv; }
+        my_v = v;
     }
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
     const float p = (lane < c.k) ? expf(my_v - vmax) : 0.f;
