@@ -48,6 +48,13 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
     return t;
 }
 
+// *p += {a, b, c, d} as one fp32 vector reduction in L2 (p 16-byte aligned; each element added
+// atomically, no ordering among them).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
     if (status) atomicOr(status, bit);
 }

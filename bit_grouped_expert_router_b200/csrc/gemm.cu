@@ -28,9 +28,12 @@
 //                    to the expert's act rows (only the tile's valid tokens).
 //   down kernel    : per tile (expert, 128 output rows, <=256 tokens), K = I.  B = act rows.
 //                    Epilogue: y * gate (routing gate, or sigmoid gate for the shared expert) added
-//                    into the token's fp32 accumulator row with coalesced red.global.add.f32 (a warp
-//                    covers 32 consecutive rows = 128 contiguous bytes of one token's row; L2 takes
-//                    such reductions at ~5 TB/s on this part, twice the rate of bulk reductions).
+//                    into the token's fp32 accumulator row.  A warp's 32 x 32 block (32 output
+//                    rows = TMEM lanes, 32 tokens) is transposed through shared memory so that each
+//                    lane adds 4 consecutive rows of one token with one red.global.add.v4.f32 (8
+//                    lanes cover a token's 128 contiguous bytes): a quarter of the reduction
+//                    instructions of one scalar red per element, which made the down GEMM ~30 %
+//                    faster on this part (the scalar form was bound by the epilogue's issue).
 //
 // Warp roles (576 threads, one persistent CTA per SM, tiles taken round-robin from the device-
 // built tile list so no tile count ever travels to the host):
@@ -80,13 +83,14 @@ constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kAS * kATileBytes;
 constexpr int kOffW = kOffB + kBS * kBTileBytes;
 constexpr int kOffStage = kOffW + kWS * kWStageBytes;
-constexpr int kStageBytes = kBN * 128;      // gate/up: kBN x 64 fp16 act staging
+constexpr int kStageBytes = kBN * 128;      // gate/up: kBN x 64 fp16 act; down: 32 x 32 fp32 per epilogue warp
 constexpr int kOffMeta = kOffStage + kStageBytes;
 constexpr int kMetaBytes = 2 * kBN * 16;    // [2 buffers][kBN] row pointer + gate (+ pad)
 constexpr int kOffBar = kOffMeta + kMetaBytes;
 constexpr int kNumBars = 2 * (kWS + kBS + kAS) + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+static_assert(kStageBytes >= kEpiWarps * 32 * 32 * 4, "down epilogue: one 32 x 32 fp32 block per warp");
 static_assert(kOffB % 1024 == 0 && kOffW % 16 == 0 && kOffStage % 16 == 0 && kOffMeta % 16 == 0 &&
                   kOffBar % 8 == 0,
               "align");
@@ -365,19 +369,27 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                 }
                 named_bar(1, 32 * kEpiWarps);
             } else {
-                const int hl = 32 * q + lane;   // output row inside the m-tile
+                // tr[r][l] = accumulator (row 32q + l, token c0 + r); lane l then reads rows
+                // 32q + 4(l % 8) .. +3 of token c0 + 4g + l / 8 as one float4
+                float* tr = reinterpret_cast<float*>(stage) + (warp - kEpiWarp0) * 1024;
+                const int h4 = 32 * q + 4 * (lane & 7);   // first of this lane's 4 output rows
                 for (int c0 = 32 * eh; c0 < nvalid; c0 += 64) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
 #pragma unroll
-                    for (int r = 0; r < 32; ++r) {
-                        const int j = c0 + r;
+                    for (int r = 0; r < 32; ++r) tr[r * 32 + lane] = __uint_as_float(v[r]);
+                    __syncwarp();
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const int jl = 4 * g + (lane >> 3);
+                        const int j = c0 + jl;
                         if (j < nvalid) {
-                            float* dst = meta_row[ab * kBN + j] + hl;
-                            const float y = __uint_as_float(v[r]) * meta_gate[ab * kBN + j];
-                            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst), "f"(y) : "memory");
+                            const float4 y = *reinterpret_cast<const float4*>(tr + jl * 32 + 4 * (lane & 7));
+                            const float gt = meta_gate[ab * kBN + j];
+                            red_add_v4(meta_row[ab * kBN + j] + h4, y.x * gt, y.y * gt, y.z * gt, y.w * gt);
                         }
                     }
+                    __syncwarp();   // tr is rewritten by the next chunk
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -408,7 +420,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(Ctx c) {
         }
         const uint4* src = reinterpret_cast<const uint4*>(c.x16 + (size_t)t * c.H);
         uint4* dst = reinterpret_cast<uint4*>(c.xp + (size_t)p * c.H);
-        for (int i = lane; i < c.H / 8; i += 32) dst[i] = src[i];
+        const int n16 = c.H / 8;
+        for (int i0 = 0; i0 < n16; i0 += 32 * 8) {   // 8 loads in flight per lane before the stores
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + 32 * u + lane;
+                if (i < n16) v[u] = src[i];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + 32 * u + lane;
+                if (i < n16) dst[i] = v[u];
+            }
+        }
     }
 }
 

@@ -325,26 +325,40 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
     }
     __syncthreads();
     if (warp == 0) {
+        // entries in (token, slot) order, 32 per step so equal experts keep that order (stable);
+        // the expert ids and gates of 16 steps are loaded before those steps run
+        constexpr int kChunk = 16;
         const int n_entries = nt * c.k;
-        for (int base = 0; base < n_entries; base += 32) {
-            const int i = base + lane;
-            const bool active = i < n_entries;
-            const int flat = t0 * c.k + i;
-            int e = active ? c.idx[flat] : -1;
-            if (active && (e < 0 || e >= c.E)) { set_status(c.status, MOE_STATUS_BOUNDS); e = 0; }
-            const unsigned mask = __match_any_sync(0xffffffffu, e);
-            const int rank = __popc(mask & ((1u << lane) - 1u));
-            const int p = active ? cnt[e] + rank : 0;
-            __syncwarp();
-            if (active && lane == __ffs(mask) - 1) cnt[e] += __popc(mask);
-            __syncwarp();
-            if (active) {
-                if (p < 0 || p >= c.rows_cap) {
-                    set_status(c.status, MOE_STATUS_BOUNDS);
-                } else {
-                    c.perm[p] = flat;
-                    c.row_token[p] = flat / c.k;
-                    c.row_gate[p] = c.gates[flat];
+        for (int base0 = 0; base0 < n_entries; base0 += 32 * kChunk) {
+            int ev[kChunk];
+            float gv[kChunk];
+#pragma unroll
+            for (int u = 0; u < kChunk; ++u) {
+                const int i = base0 + 32 * u + lane;
+                ev[u] = i < n_entries ? c.idx[t0 * c.k + i] : -1;
+                gv[u] = i < n_entries ? c.gates[t0 * c.k + i] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kChunk; ++u) {
+                const int i = base0 + 32 * u + lane;
+                const bool active = i < n_entries;
+                const int flat = t0 * c.k + i;
+                int e = ev[u];
+                if (active && (e < 0 || e >= c.E)) { set_status(c.status, MOE_STATUS_BOUNDS); e = 0; }
+                const unsigned mask = __match_any_sync(0xffffffffu, e);
+                const int rank = __popc(mask & ((1u << lane) - 1u));
+                const int p = active ? cnt[e] + rank : 0;
+                __syncwarp();
+                if (active && lane == __ffs(mask) - 1) cnt[e] += __popc(mask);
+                __syncwarp();
+                if (active) {
+                    if (p < 0 || p >= c.rows_cap) {
+                        set_status(c.status, MOE_STATUS_BOUNDS);
+                    } else {
+                        c.perm[p] = flat;
+                        c.row_token[p] = flat / c.k;
+                        c.row_gate[p] = gv[u];
+                    }
                 }
             }
         }
