@@ -87,7 +87,7 @@ Layout make_layout(const moe_config& c) {
     L.ks_dec = c.hidden / kRouterKSlice;
     L.nblk_max = (L.Tm + kTokPerBucketBlk - 1) / kTokPerBucketBlk;
     L.rows_cap = L.Tm * L.k + (c.has_shared ? L.Tm : 0);
-    L.max_tiles = (L.rows_cap + kBN - 1) / kBN + L.G;
+    L.max_tiles = (L.rows_cap + 127) / 128 + L.G;   // tiles of >= 128 rows (gemm_tile_rows)
     const size_t per_mat_gu = (size_t)(L.I / 64) * (L.H / 64) * kBlockBytes;   // gate+up rows 2I
     const size_t per_mat_dn = (size_t)(L.H / 128) * (L.I / 64) * kBlockBytes;
     L.w_gu_bytes = per_mat_gu * L.G;
@@ -229,6 +229,7 @@ namespace {
 Ctx make_ctx(const moe_handle* h, int T, const uint16_t* x, uint16_t* out, bool decode) {
     Ctx c = h->base;
     c.T = T;
+    c.tile_rows = gemm_tile_rows(T, c.k, c.E);
     c.x = x;
     c.out = out;
     c.nblk = (T + kTokPerBucketBlk - 1) / kTokPerBucketBlk;

@@ -35,15 +35,17 @@
 //                    instructions of one scalar red per element, which made the down GEMM ~30 %
 //                    faster on this part (the scalar form was bound by the epilogue's issue).
 //
-// Warp roles (576 threads, one persistent CTA per SM, tiles taken round-robin from the device-
-// built tile list so no tile count ever travels to the host):
+// Warp roles (one persistent CTA per SM with 576 threads and 256-token tiles, or two per SM with
+// 320 threads and 128-token tiles -- GemmCfg; tiles taken round-robin from the device-built tile
+// list so no tile count ever travels to the host):
 //   warp 0      TMA producer (lane 0)
 //   warp 1      TMEM allocator + MMA issuer (one lane)
-//   warps 2-9   transform: dequantise a block into the A ring (thread = row, half of 64 columns)
-//   warps 10-17 epilogue: drain a TMEM accumulator (double-buffered, so it overlaps the next tile;
-//               warp w reads TMEM lanes 32*(w%4)..+31, the two warps of a lane quarter take
-//               alternate 32-column chunks)
-// TMEM: two 256-column fp32 accumulators.  Every wait is bounded (common.cuh); on a timeout the
+//   transform   warps 2-9 (or 2-5): dequantise a block into the A ring (thread = row, half of the
+//               64 columns; both halves with 4 warps)
+//   epilogue    warps 10-17 (or 6-9): drain a TMEM accumulator (double-buffered, so it overlaps
+//               the next tile; warp w reads TMEM lanes 32*(w%4)..+31, the warps of a lane quarter
+//               take alternate 32-column chunks)
+// TMEM: two fp32 accumulators of kBN columns.  Every wait is bounded (common.cuh); on a timeout the
 // roles unwind, the producer waits for its copies in flight, the MMA thread waits for its MMAs,
 // and warp 1 frees the TMEM.
 #include "common.cuh"
@@ -53,57 +55,65 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 576;
-constexpr int kEpiWarps = 8;
-constexpr int kTransformWarps = 8;
-constexpr int kEpiWarp0 = 2 + kTransformWarps;
-constexpr int kTmemCols = 512;
-constexpr int kAccCols = kBN;
-static_assert(2 * kAccCols <= kTmemCols, "TMEM budget");
-static_assert(kBN == 256, "token tile");
-
-#ifndef GEMM_KWB
-#define GEMM_KWB 4
-#endif
-constexpr int kWB = GEMM_KWB;   // weight blocks per bulk copy
-constexpr int kWS = 2;   // weight ring stages
-#ifndef GEMM_KBS
-#define GEMM_KBS 3
-#endif
-#ifndef GEMM_KAS
-#define GEMM_KAS 3
-#endif
-constexpr int kBS = GEMM_KBS;   // token ring stages
-constexpr int kAS = GEMM_KAS;   // A ring stages
-
-constexpr int kATileBytes = 128 * 128;      // 128 weight rows x 64 fp16
-constexpr int kBTileBytes = kBN * 128;      // up to 256 token rows x 64 fp16
-constexpr int kWStageBytes = kWB * kBlockBytes;
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kAS * kATileBytes;
-constexpr int kOffW = kOffB + kBS * kBTileBytes;
-constexpr int kOffStage = kOffW + kWS * kWStageBytes;
-constexpr int kStageBytes = kBN * 128;      // gate/up: kBN x 64 fp16 act; down: 32 x 32 fp32 per epilogue warp
-constexpr int kOffMeta = kOffStage + kStageBytes;
-constexpr int kMetaBytes = 2 * kBN * 16;    // [2 buffers][kBN] row pointer + gate (+ pad)
-constexpr int kOffBar = kOffMeta + kMetaBytes;
-constexpr int kNumBars = 2 * (kWS + kBS + kAS) + 5;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-static_assert(kStageBytes >= kEpiWarps * 32 * 32 * 4, "down epilogue: one 32 x 32 fp32 block per warp");
-static_assert(kOffB % 1024 == 0 && kOffW % 16 == 0 && kOffStage % 16 == 0 && kOffMeta % 16 == 0 &&
-                  kOffBar % 8 == 0,
-              "align");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+// Two launch shapes of the same kernel.  CTAS = 1: one 576-thread CTA per SM, 256-token tiles,
+// rings of 3 token / 3 A stages and 4-block weight copies.  CTAS = 2: two 320-thread CTAs per SM
+// (half the roles and half the TMEM each), 128-token tiles, 2 + 2 stages and 2-block copies.  The
+// MMA-issuing thread's chain of waits, issues and commits bounds a k-step at ~1000 cycles whatever
+// the tile's token count, so when experts get few tokens (tiles far from full) two independent
+// chains per SM win; when tiles are full, the larger tile's fewer k-steps win (host picks per call).
+template <int CTAS>
+struct GemmCfg {
+    static_assert(CTAS == 1 || CTAS == 2, "CTAs per SM");
+    static constexpr int kBN = CTAS == 1 ? 256 : 128;   // token columns per tile (= UMMA N)
+    static constexpr int kEpiWarps = 8 / CTAS;
+    static constexpr int kTransformWarps = 8 / CTAS;
+    static constexpr int kEpiWarp0 = 2 + kTransformWarps;
+    static constexpr int kThreads = 32 * (2 + kTransformWarps + kEpiWarps);
+    static constexpr int kTmemCols = 512 / CTAS;
+    static constexpr int kAccCols = kBN;
+    static constexpr int kWB = CTAS == 1 ? 4 : 2;   // weight blocks per bulk copy
+    static constexpr int kWS = 2;                   // weight ring stages
+    static constexpr int kBS = CTAS == 1 ? 3 : 2;   // token ring stages
+    static constexpr int kAS = CTAS == 1 ? 3 : 2;   // A ring stages
+    static constexpr int kATileBytes = 128 * 128;   // 128 weight rows x 64 fp16
+    static constexpr int kBTileBytes = kBN * 128;   // up to kBN token rows x 64 fp16
+    static constexpr int kWStageBytes = kWB * kBlockBytes;
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kOffA + kAS * kATileBytes;
+    static constexpr int kOffW = kOffB + kBS * kBTileBytes;
+    static constexpr int kOffStage = kOffW + kWS * kWStageBytes;
+    static constexpr int kStageBytes = kBN * 128;   // gate/up: kBN x 64 fp16 act; down: 32 x 32 fp32 per epilogue warp
+    static constexpr int kOffMeta = kOffStage + kStageBytes;
+    static constexpr int kMetaBytes = 2 * kBN * 16; // [2 buffers][kBN] row pointer + gate (+ pad)
+    static constexpr int kOffBar = kOffMeta + kMetaBytes;
+    static constexpr int kNumBars = 2 * (kWS + kBS + kAS) + 5;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    static_assert(kBN <= moe::kBN, "tile lists are sized for at most kBN rows per tile");
+    static_assert(2 * kAccCols <= kTmemCols, "TMEM budget");
+    static_assert(kStageBytes >= kEpiWarps * 32 * 32 * 4, "down epilogue: one 32 x 32 fp32 block per warp");
+    static_assert(kOffB % 1024 == 0 && kOffW % 16 == 0 && kOffStage % 16 == 0 && kOffMeta % 16 == 0 &&
+                      kOffBar % 8 == 0,
+                  "align");
+    static_assert(kSmemBytes * CTAS <= 227 * 1024, "shared memory budget");
+};
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g * u / (1.f + __expf(-g)); }
 
-__device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c) {
-    return t.x >= 0 && t.x < c.G && t.y >= 0 && t.z > 0 && t.z <= kBN && t.y + t.z <= c.rows_cap;
+__device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c, int bn) {
+    return t.x >= 0 && t.x < c.G && t.y >= 0 && t.z > 0 && t.z <= bn && t.y + t.z <= c.rows_cap;
 }
 
-template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps) {
+template <bool GATEUP, int CTAS>
+__global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
+    grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps) {
+    using K = GemmCfg<CTAS>;
+    constexpr int kBN = K::kBN, kEpiWarps = K::kEpiWarps, kTransformWarps = K::kTransformWarps;
+    constexpr int kEpiWarp0 = K::kEpiWarp0, kTmemCols = K::kTmemCols, kAccCols = K::kAccCols;
+    constexpr int kWB = K::kWB, kWS = K::kWS, kBS = K::kBS, kAS = K::kAS;
+    constexpr int kATileBytes = K::kATileBytes, kBTileBytes = K::kBTileBytes, kWStageBytes = K::kWStageBytes;
+    constexpr int kOffA = K::kOffA, kOffB = K::kOffB, kOffW = K::kOffW, kOffStage = K::kOffStage;
+    constexpr int kOffMeta = K::kOffMeta, kOffBar = K::kOffBar, kOffMisc = K::kOffMisc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* asm_ = smem + kOffA;
@@ -175,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
                 const int mt = tau % MT;
-                if (!tile_ok(tile, c)) continue;
+                if (!tile_ok(tile, c, kBN)) continue;
                 const int n_inst = max(16, ((tile.z + 15) / 16) * 16);
                 const int hsel = n_inst <= 64 ? 0 : (n_inst <= 128 ? 1 : 2);
                 const bool from_x = GATEUP && c.has_shared && tile.x == c.E;   // shared expert: token order
@@ -228,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
             const uint32_t a0 = smem_u32(asm_), b0 = smem_u32(bsm);
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
-                if (!tile_ok(tile, c)) {
+                if (!tile_ok(tile, c, kBN)) {
                     if (tau % MT == 0) set_status(c.status, MOE_STATUS_BOUNDS);
                     continue;
                 }
@@ -264,22 +274,26 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------------ transform
-        // thread = (weight row, half of the 64 columns); the fp16 pairs of 16-byte chunk ch of row r
-        // go to r*128 + ((ch ^ (r & 7)) * 16), the 128-byte swizzle the MMA descriptor expects.
-        const int tt = threadIdx.x - 64;        // 0..255
-        const int row = tt & 127, half = tt >> 7;
+        // thread = (weight row, half of the 64 columns; both halves when there are 4 transform
+        // warps); the fp16 pairs of 16-byte chunk ch of row r go to r*128 + ((ch ^ (r & 7)) * 16),
+        // the 128-byte swizzle the MMA descriptor expects.
+        const int tt = threadIdx.x - 64;        // 0 .. 32 * kTransformWarps - 1
+        const int row = tt & 127;
         const uint32_t sw = (uint32_t)(row & 7);
         int ws = 0, as = 0;
         uint32_t wph = 0, aph = 0;
         for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
             const int4 tile = c.tiles1[tau / MT];
-            if (!tile_ok(tile, c)) continue;
+            if (!tile_ok(tile, c, kBN)) continue;
             for (int kc = 0; kc < KS; ++kc) {
                 // waits end the same way for the whole warp (the vote), so no lane is left behind
                 bool ok = kc % kWB != 0 || mbar_wait(&wfull[ws], wph, abort_flag, c.status);
                 ok = ok && mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status);
                 if (!__all_sync(0xffffffffu, ok)) goto transform_done;
                 const uint8_t* blk = wsm + ws * kWStageBytes + (kc % kWB) * kBlockBytes;
+#pragma unroll
+                for (int hi = 0; hi < 8 / kTransformWarps; ++hi) {
+                const int half = kTransformWarps == 8 ? (tt >> 7) : hi;
                 const uint4 cw = *reinterpret_cast<const uint4*>(blk + half * 2048 + row * 16);
                 const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
                 const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)),
@@ -299,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                     const uint32_t ch = (uint32_t)(4 * half + w);
                     *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(r[0], r[1], r[2], r[3]);
                 }
+                }
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&afull[as]);
@@ -313,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;
-        const int eh = (warp - kEpiWarp0) >> 2;           // which of the two warps of this quarter
+        const int eh = (warp - kEpiWarp0) >> 2;           // which of this quarter's warps (0 or 0/1)
         const int etid = threadIdx.x - 32 * kEpiWarp0;   // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint32_t tl = 0;
@@ -321,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
         for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
             const int4 tile = c.tiles1[tau / MT];
             const int mt = tau % MT;
-            if (!tile_ok(tile, c)) continue;
+            if (!tile_ok(tile, c, kBN)) continue;
             const int row0 = tile.y, nvalid = tile.z;
             const uint32_t ab = tl & 1u, aph = (tl >> 1) & 1u;
             ++tl;
@@ -341,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
             if (GATEUP) {
                 const int ilocal = 16 * q + (lane & 15);
                 const bool is_gate = lane < 16;
-                for (int c0 = 32 * eh; c0 < nvalid; c0 += 64) {
+                for (int c0 = 32 * eh; c0 < nvalid; c0 += 32 * (kEpiWarps / 4)) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
 #pragma unroll
@@ -373,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Ctx c, const 
                 // 32q + 4(l % 8) .. +3 of token c0 + 4g + l / 8 as one float4
                 float* tr = reinterpret_cast<float*>(stage) + (warp - kEpiWarp0) * 1024;
                 const int h4 = 32 * q + 4 * (lane & 7);   // first of this lane's 4 output rows
-                for (int c0 = 32 * eh; c0 < nvalid; c0 += 64) {
+                for (int c0 = 32 * eh; c0 < nvalid; c0 += 32 * (kEpiWarps / 4)) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
 #pragma unroll
@@ -439,7 +454,21 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(Ctx c) {
 
 }  // namespace
 
-int gemm_smem_bytes(bool) { return kSmemBytes; }
+namespace {
+
+template <bool GATEUP, int CTAS>
+cudaError_t launch_grouped(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
+    using K = GemmCfg<CTAS>;
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, CTAS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    grouped_gemm_kernel<GATEUP, CTAS><<<num_sms * CTAS, K::kThreads, K::kSmemBytes, st>>>(c, maps);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_tile_rows(int T, int k, int E) { return T * k <= 64 * E ? GemmCfg<2>::kBN : GemmCfg<1>::kBN; }
 
 cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st) {
     const int rows = c.T * c.k;
@@ -448,20 +477,17 @@ cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// The tile list (built for c.tile_rows rows per tile) selects the launch shape.
 cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<true><<<num_sms, kThreads, kSmemBytes, st>>>(c, maps);
-    return cudaGetLastError();
+    if (c.tile_rows == GemmCfg<2>::kBN) return launch_grouped<true, 2>(c, maps, num_sms, st);
+    if (c.tile_rows == GemmCfg<1>::kBN) return launch_grouped<true, 1>(c, maps, num_sms, st);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<false><<<num_sms, kThreads, kSmemBytes, st>>>(c, maps);
-    return cudaGetLastError();
+    if (c.tile_rows == GemmCfg<2>::kBN) return launch_grouped<false, 2>(c, maps, num_sms, st);
+    if (c.tile_rows == GemmCfg<1>::kBN) return launch_grouped<false, 1>(c, maps, num_sms, st);
+    return cudaErrorInvalidValue;
 }
 
 // out[t][h] = bf16(acc[t][h]), round to nearest even; 8 elements per thread per step.

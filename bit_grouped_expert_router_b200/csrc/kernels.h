@@ -9,7 +9,7 @@
 namespace moe {
 
 // Tile geometry of the prefill grouped GEMMs (tokens per tile = UMMA N).
-constexpr int kBN = 256;          // token columns per tile (= UMMA N)
+constexpr int kBN = 256;          // largest token tile of the grouped GEMMs (= UMMA N); tile lists are sized by 128
 constexpr int kStages = 3;        // pipeline depth (shared-memory stages)
 constexpr int kTokPerBucketBlk = 64;  // tokens per routing/bucketing CTA
 constexpr int kRouterTT = 32;     // tokens per CTA in the SIMT router (prefill sizes)
@@ -48,6 +48,7 @@ struct Ctx {
     int nblk;          // routing/bucketing CTAs for T tokens
     int ks;            // K slices of the router partial logits
     int max_tiles;     // capacity of each tile list
+    int tile_rows;     // token rows per grouped-GEMM tile (128 or 256), set per call
     int rows_cap;      // row capacity of xp / act
     uint32_t flags;
     // weights, kernel layout
@@ -112,7 +113,9 @@ cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st);
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st);
-int gemm_smem_bytes(bool gateup);
+// Token rows per grouped-GEMM tile for a call of T tokens: 128 (two CTAs per SM) when the
+// routed experts average at most 64 tokens (T * k <= 64 * E), else 256 (one CTA per SM).
+int gemm_tile_rows(int T, int k, int E);
 
 // host-side error text for moe_last_error() (defined in api.cu)
 void set_last_error(const char* msg);

@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
         for (int base = 0; base < c.G; base += 32) {
             const int g = base + lane;
             const int v = (g < c.G) ? cnt[g] : 0;
-            const int nt = (v + kBN - 1) / kBN;
+            const int nt = (v + c.tile_rows - 1) / c.tile_rows;
             const int inc = warp_incl_scan(v);
             const int tinc = warp_incl_scan(nt);
             if (g < c.G) { off[g] = run + inc - v; toff[g] = trun + tinc - nt; }
@@ -299,8 +299,8 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
     for (int g = tid; g < c.G; g += blockDim.x) {
         const int n = cnt[g];
         int tslot = toff[g];
-        for (int n0 = 0; n0 < n; n0 += kBN, ++tslot) {
-            if (tslot < c.max_tiles) c.tiles1[tslot] = make_int4(g, off[g] + n0, min(kBN, n - n0), 0);
+        for (int n0 = 0; n0 < n; n0 += c.tile_rows, ++tslot) {
+            if (tslot < c.max_tiles) c.tiles1[tslot] = make_int4(g, off[g] + n0, min(c.tile_rows, n - n0), 0);
             else set_status(c.status, MOE_STATUS_BOUNDS);
         }
     }
