@@ -509,7 +509,9 @@ __global__ void __launch_bounds__(256) finalize_kernel(Ctx c) {
 
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st) {
     const size_t n8 = (size_t)c.T * c.H / 8;
-    const int blocks = (int)((n8 + 255) / 256 < 148 * 8 ? (n8 + 255) / 256 : 148 * 8);
+    // one 8-element chunk per thread (the loop only covers grids past the launch limit)
+    const size_t want = (n8 + 255) / 256;
+    const int blocks = (int)(want < (size_t)(1u << 30) ? want : (size_t)(1u << 30));
     finalize_kernel<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(c);
     return cudaGetLastError();
 }

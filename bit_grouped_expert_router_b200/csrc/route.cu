@@ -184,27 +184,38 @@ __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
     float d = 0.f;
     bool range_bad = false;
     if (c.has_shared || do_hist) {
-        for (int h = lane * 8; h < c.H; h += 256) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(xr + h);
-            if (c.has_shared) {
-                const float4 w0 = *reinterpret_cast<const float4*>(c.sgw + h);
-                const float4 w1 = *reinterpret_cast<const float4*>(c.sgw + h + 4);
-                d = fmaf(__uint_as_float(raw.x << 16), w0.x, d);
-                d = fmaf(__uint_as_float(raw.x & 0xFFFF0000u), w0.y, d);
-                d = fmaf(__uint_as_float(raw.y << 16), w0.z, d);
-                d = fmaf(__uint_as_float(raw.y & 0xFFFF0000u), w0.w, d);
-                d = fmaf(__uint_as_float(raw.z << 16), w1.x, d);
-                d = fmaf(__uint_as_float(raw.z & 0xFFFF0000u), w1.y, d);
-                d = fmaf(__uint_as_float(raw.w << 16), w1.z, d);
-                d = fmaf(__uint_as_float(raw.w & 0xFFFF0000u), w1.w, d);
-            }
-            if (do_hist) {   // fp16 copy of the row for the tensor-core path (exact for |x| < 65504)
-                uint4 o;
-                o.x = bf16x2_to_half2_bits(raw.x, &range_bad);
-                o.y = bf16x2_to_half2_bits(raw.y, &range_bad);
-                o.z = bf16x2_to_half2_bits(raw.z, &range_bad);
-                o.w = bf16x2_to_half2_bits(raw.w, &range_bad);
-                *reinterpret_cast<uint4*>(c.x16 + (size_t)t * c.H + h) = o;
+        // the lane's row loads (up to 8 chunks of 8 elements) are all issued before the arithmetic
+        constexpr int kXU = 8;
+        for (int h0 = lane * 8; h0 < c.H; h0 += 256 * kXU) {
+            uint4 rawv[kXU];
+#pragma unroll
+            for (int u = 0; u < kXU; ++u)
+                if (h0 + 256 * u < c.H) rawv[u] = __ldg(reinterpret_cast<const uint4*>(xr + h0 + 256 * u));
+#pragma unroll
+            for (int u = 0; u < kXU; ++u) {
+                const int h = h0 + 256 * u;
+                if (h >= c.H) break;
+                const uint4 raw = rawv[u];
+                if (c.has_shared) {
+                    const float4 w0 = *reinterpret_cast<const float4*>(c.sgw + h);
+                    const float4 w1 = *reinterpret_cast<const float4*>(c.sgw + h + 4);
+                    d = fmaf(__uint_as_float(raw.x << 16), w0.x, d);
+                    d = fmaf(__uint_as_float(raw.x & 0xFFFF0000u), w0.y, d);
+                    d = fmaf(__uint_as_float(raw.y << 16), w0.z, d);
+                    d = fmaf(__uint_as_float(raw.y & 0xFFFF0000u), w0.w, d);
+                    d = fmaf(__uint_as_float(raw.z << 16), w1.x, d);
+                    d = fmaf(__uint_as_float(raw.z & 0xFFFF0000u), w1.y, d);
+                    d = fmaf(__uint_as_float(raw.w << 16), w1.z, d);
+                    d = fmaf(__uint_as_float(raw.w & 0xFFFF0000u), w1.w, d);
+                }
+                if (do_hist) {   // fp16 copy of the row for the tensor-core path (exact for |x| < 65504)
+                    uint4 o;
+                    o.x = bf16x2_to_half2_bits(raw.x, &range_bad);
+                    o.y = bf16x2_to_half2_bits(raw.y, &range_bad);
+                    o.z = bf16x2_to_half2_bits(raw.z, &range_bad);
+                    o.w = bf16x2_to_half2_bits(raw.w, &range_bad);
+                    *reinterpret_cast<uint4*>(c.x16 + (size_t)t * c.H + h) = o;
+                }
             }
         }
     }
