@@ -174,6 +174,22 @@ def test_full_decode_workload(layer_idx):
     layer2.close()
 
 
+def test_both_grouped_gemm_launch_shapes_around_the_switch():
+    """The grouped GEMMs run as two CTAs per SM with 128-token tiles while T * k <= 64 * E and as
+    one CTA per SM with 256-token tiles above: T = 2048 and 2049 at the full layer sizes sit on
+    either side of the switch (same layer, same leading tokens)."""
+    shape = synth.Shape("switch", T=2049, H=2048, E=256, k=8, I=512, zipf_s=1.1, seed=32)
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=16)
+    for T in (2048, 2049):
+        sub = synth.shape_with(shape, T=T)
+        _route_check(layer, ol, x[:T], sub)
+        print("T =", T, _forward_check(layer, ol, x[:T], tokens=_sample(T, 96, 5)))
+    layer.close()
+
+
 def test_forced_experts_make_large_buckets():
     shape = synth.Shape("forced", T=1024, H=2048, E=256, k=8, I=512, seed=31)
     w = synth.make_layer(shape)
