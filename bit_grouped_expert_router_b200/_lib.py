@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
                                  ctypes.POINTER(P)]
         L.moe_forward.argtypes = [P, P, I32, P, P]
         L.moe_forward_host.argtypes = [P, P, I32, P, P]
+        L.moe_forward_host_async.argtypes = [P, P, I32, P, P]
         L.moe_route.argtypes = [P, P, I32, P, P, P, P, P, P]
         L.moe_status.argtypes = [P]
         L.moe_debug_copy.argtypes = [P, ctypes.c_int, P, SZ, P]
@@ -81,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_enable.argtypes = [P, ctypes.c_int]
         L.moe_profile_read.argtypes = [P, P, P]
         L.moe_route_static.argtypes = [P, I32, I32, P, P, I32, I32, P, P, P]
-        for n in ("moe_create", "moe_forward", "moe_forward_host", "moe_route", "moe_status",
+        for n in ("moe_create", "moe_forward", "moe_forward_host", "moe_forward_host_async", "moe_route", "moe_status",
                   "moe_debug_copy", "moe_profile_enable", "moe_profile_read", "moe_route_static"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
@@ -163,6 +164,13 @@ class Layer:
         if out_host is None:
             out_host = torch.empty((T, self.H), dtype=torch.bfloat16, pin_memory=True)
         check(lib().moe_forward_host(self.handle, _ptr(x_host), T, _ptr(out_host), _stream_ptr(stream)))
+        return out_host
+
+    def forward_host_async(self, x_host, out_host, stream=None):
+        """Enqueue copy-in, layer and copy-out on `stream` and return; `out_host` is valid once the
+        stream has passed this call (pinned host tensors give overlapped copies)."""
+        check(lib().moe_forward_host_async(self.handle, _ptr(x_host), x_host.shape[0], _ptr(out_host),
+                                           _stream_ptr(stream)))
         return out_host
 
     def route(self, x, stream=None):

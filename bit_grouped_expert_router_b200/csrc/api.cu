@@ -496,7 +496,7 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     return MOE_OK;
 }
 
-int moe_forward_host(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t* out_host, void* stream) {
+int moe_forward_host_async(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t* out_host, void* stream) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
     if (T > h->cfg.max_tokens) return fail(MOE_ERR_TOO_LARGE, "T = %d exceeds max_tokens = %d", T, h->cfg.max_tokens);
@@ -511,7 +511,14 @@ int moe_forward_host(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t*
     int rc = moe_forward(h, dx, T, dout, stream);
     if (rc != MOE_OK) return rc;
     CUDA_TRY(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st));
-    CUDA_TRY(cudaStreamSynchronize(st));
+    return MOE_OK;
+}
+
+int moe_forward_host(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t* out_host, void* stream) {
+    const int rc = moe_forward_host_async(h, x_host, T, out_host, stream);
+    if (rc != MOE_OK || T == 0) return rc;
+    DeviceGuard guard(h->device);
+    CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     return MOE_OK;
 }
 

@@ -23,15 +23,16 @@
  * library's layer definition; the pages do not spell them out.
  *
  * Conventions for every entry point below.
- *  - All tensor pointers are DEVICE pointers owned by the caller (except moe_forward_host, which
- *    takes host pointers).  The library never frees or retains caller memory beyond the call,
- *    except that moe_create copies (repacks) the weights into memory the handle owns, so the
- *    caller may free its weight buffers as soon as moe_create has returned and its stream has
- *    been synchronised.
+ *  - All tensor pointers are DEVICE pointers owned by the caller (except moe_forward_host and
+ *    moe_forward_host_async, which take host pointers).  The library never frees or retains
+ *    caller memory beyond the call, except that moe_create copies (repacks) the weights into
+ *    memory the handle owns, so the caller may free its weight buffers as soon as moe_create has
+ *    returned and its stream has been synchronised.
  *  - "stream" is a cudaStream_t passed as void* (NULL = the legacy default stream).  Calls are
  *    stream-ordered and asynchronous: they return after enqueueing work, with no host
  *    synchronisation, no device-to-host copy and no allocation (moe_create and moe_forward_host
- *    excepted).  Outputs are overwritten, never accumulated into.
+ *    excepted; moe_forward_host_async enqueues its device-to-host copy without waiting for it).
+ *    Outputs are overwritten, never accumulated into.
  *  - Return value: MOE_OK or one of the MOE_ERR_* codes.  No exception crosses the ABI.  An error
  *    found before launch returns its code and launches nothing; a text message is then available
  *    from moe_last_error() on the calling thread.  Errors found on the device (a timed-out wait,
@@ -131,6 +132,17 @@ MOE_API int moe_forward(moe_handle *h, const uint16_t *x, int32_t T, uint16_t *o
  * fastest; pageable memory works.  Uses handle-owned device staging buffers (no allocation). */
 MOE_API int moe_forward_host(moe_handle *h, const uint16_t *x_host, int32_t T, uint16_t *out_host,
                      void *stream);
+
+/* moe_forward_host without the final synchronisation: the copy in, the layer and the copy out are
+ * enqueued on `stream` and the call returns.  x_host must stay unchanged and out_host unread until
+ * the stream has passed the copy out (synchronise the stream or an event recorded after the call).
+ * With pinned host memory the copies are asynchronous, so calls on different handles issued to
+ * different streams overlap one layer's copies with another's kernels; pageable memory works but
+ * its copies are staged through the driver and overlap little.  The handle's staging buffers are
+ * reused by its next call, which is safe because calls on one handle are ordered on its stream.
+ * Errors: as moe_forward_host (before launch), device errors via moe_status. */
+MOE_API int moe_forward_host_async(moe_handle *h, const uint16_t *x_host, int32_t T, uint16_t *out_host,
+                           void *stream);
 
 /* Routing and bucketing only (the first steps of the prefill path), with their results copied
  * to caller device buffers (any output pointer may be NULL to skip it):

@@ -17,7 +17,8 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = M.header_functions()
-    assert set(names) >= {"moe_create", "moe_forward", "moe_forward_host", "moe_route", "moe_status",
+    assert set(names) >= {"moe_create", "moe_forward", "moe_forward_host", "moe_forward_host_async",
+                          "moe_route", "moe_status",
                           "moe_debug_copy", "moe_device_bytes", "moe_last_error", "moe_destroy",
                           "moe_version"}
     for n in names:
@@ -69,6 +70,7 @@ def test_null_handle_calls(lib):
     assert lib.moe_route(None, None, 1, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_status(None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_forward_host(None, None, 1, None, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host_async(None, None, 1, None, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_copy(None, 0, None, 0, None) == M.MOE_ERR_INVALID_ARG
     lib.moe_destroy(None)
 

@@ -216,6 +216,20 @@ def test_host_buffers_and_edge_calls():
     dev = layer.forward(x.cuda()).cpu()
     host = layer.forward_host(x.pin_memory())
     assert torch.equal(dev.view(torch.int16), host.view(torch.int16))
+    # the asynchronous variant: two handles on two streams, calls enqueued back to back
+    layer2 = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=2)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    xh = x.pin_memory()
+    outs = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+    for _ in range(3):
+        layer.forward_host_async(xh, outs[0], streams[0])
+        layer2.forward_host_async(xh, outs[1], streams[1])
+    for s in streams:
+        s.synchronize()
+    for o in outs:   # same inputs and weights: equal up to the order of the fp32 reductions
+        torch.testing.assert_close(o.float(), dev.float(), rtol=1e-2, atol=1e-2)
+    assert layer2.status() == M.MOE_OK
+    layer2.close()
     # T = 0 is a no-op, T > max_tokens is refused before launch
     assert M.lib().moe_forward(layer.handle, x.cuda().data_ptr(), 0, None, None) == M.MOE_OK
     out = torch.empty((shape.T + 1, shape.H), dtype=torch.bfloat16, device="cuda")
