@@ -269,18 +269,23 @@ def run_prefill(args, dist, peaks, peak_src):
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     if not args.no_e2e:
         xh = [[xs[l][c].cpu().pin_memory() for c in range(chunks)] for l in range(n_layers)]
-        # two streams, layer l on stream l % 2 (a handle always on the same stream): one layer's
-        # copies in and out overlap the other stream's kernels; one pinned output per stream
-        side = [torch.cuda.Stream(), torch.cuda.Stream()]
+        # one stream per prompt chunk, each chunk through the layers in order (chunked prefill);
+        # chunk c enters layer l after chunk c - 1 has left it (one event per layer handle, so a
+        # handle's workspace is never used by two streams at once): a wavefront in which one
+        # chunk's PCIe copies overlap the other chunks' kernels.  One pinned output per chunk.
+        side = [torch.cuda.Stream() for _ in range(chunks)]
+        done = [torch.cuda.Event() for _ in range(n_layers)]
         oh = [torch.empty((shape.T, shape.H), dtype=torch.bfloat16).pin_memory() for _ in side]
 
         def step_host():
             cur = torch.cuda.current_stream()
             for s in side:
                 s.wait_stream(cur)
-            for c in range(chunks):
-                for l in range(n_layers):
-                    layers[l].forward_host_async(xh[l][c], oh[l % 2], side[l % 2])
+            for l in range(n_layers):
+                for c in range(chunks):
+                    side[c].wait_event(done[l])   # (not yet recorded: no wait)
+                    layers[l].forward_host_async(xh[l][c], oh[c], side[c])
+                    done[l].record(side[c])
             for s in side:
                 cur.wait_stream(s)
         ms_e2e = timed(step_host, max(1, args.steps // 2), 1, dist)
@@ -288,7 +293,7 @@ def run_prefill(args, dist, peaks, peak_src):
         res["e2e"] = {"value": dist.world * tokens_per_step / (ms_e2e / 1000.0), "unit": "tokens/s",
                       "h2d_bytes_per_step": bytes_io, "d2h_bytes_per_step": bytes_io,
                       "ms_per_step": round(ms_e2e, 3),
-                      "api": "moe_forward_host_async (pinned host buffers, layers alternating over two streams)"}
+                      "api": "moe_forward_host_async (pinned host buffers, one stream per chunk, layer order kept)"}
         del xh
     res["host0"] = host0
     res["x0"] = xs[0][0].cpu()
