@@ -254,6 +254,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
                 prefetch_l2(c.w_gu + (((size_t)E * MTg + mt) * KSg + k0) * kBlockBytes, (uint32_t)((k1 - k0) * kBlockBytes));
         }
     }
+    // Launched as a programmatic dependent of the previous kernel in the stream: everything above
+    // reads only the handle's weights; x and the workspace are touched only after the previous
+    // grid has completed and its memory is visible.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int i = threadIdx.x; i < H; i += kFThreads) x32[i] = __uint_as_float((uint32_t)xr[i] << 16);
     if (threadIdx.x == 0) *abort_flag = 0;
     __syncthreads();
@@ -360,6 +364,9 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
         }
     }
     if (!grid_barrier(c.dfz.bar, gridDim.x, c.status, abort_flag)) return;
+    // the next kernel in the stream may be scheduled from here on (its CTAs take an SM as this
+    // grid's CTAs leave it, and wait for this grid's completion before reading anything it writes)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ------------------------------------------------------------------ phase 2: down + combine
     const int tasks_per_slot = MTd * 4 * kDnKR;
@@ -431,11 +438,13 @@ cudaError_t launch_decode_fused(const Ctx& c, int num_sms, cudaStream_t st) {
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlaps the launch with the previous kernel's tail
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, decode_fused_kernel, c);
 }
 
