@@ -467,22 +467,31 @@ def run_decode(args, dist, peaks, peak_src):
 
 
 # ------------------------------------------------------------------------------------ ncu traffic
+def kernel_code_hash():
+    """sha256 (16 hex digits) of the grouped-GEMM kernel code: csrc/gemm.cu, common.cuh and
+    kernels.h with comments and whitespace removed, concatenated (comment edits keep the hash)."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(here, "bit_grouped_expert_router_b200", "csrc", f)) as fh:
+            src = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", " ", src).strip().encode())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic(kernel):
     """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary, or None when
-    the kernel sources changed since that capture (the summary records their sha256)."""
-    import hashlib
+    the kernel code changed since that capture (the summary records kernel_code_hash())."""
     here = os.path.dirname(os.path.abspath(__file__))
     prof = os.path.join(here, "profiles", "grouped_gemm_prefill16k_zipf_1layer.md")
     if not os.path.exists(prof):
         return None
-    h = hashlib.sha256()
-    for f in ("gemm.cu", "common.cuh", "kernels.h"):
-        with open(os.path.join(here, "bit_grouped_expert_router_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
     text = open(prof).read()
     m = re.search(r"kernel_sources_sha256_16: ([0-9a-f]{16})", text)
     t = re.search(r"traffic_bytes_per_launch %s: (\d+)" % re.escape(kernel), text)
-    if not m or not t or m.group(1) != h.hexdigest()[:16]:
+    if not m or not t or m.group(1) != kernel_code_hash():
         return None
     return int(t.group(1))
 

@@ -2,31 +2,32 @@
 //
 // "Perplexity Open-Sources Lily..." section "The optimizations follow the workload": the 4-bit
 // weights are reconstructed inside the grouped matrix multiplication rather than expanded into a
-// full weight array in memory.  Here one bulk copy brings four 4608-byte blocks of packed codes +
-// fp16 scale/bias (128 weight rows x 4 x 64 input columns) into shared memory, eight "transform"
+// full weight array in memory.  Here one bulk copy brings kWB 4608-byte blocks of packed codes +
+// fp16 scale/bias (128 weight rows x kWB x 64 input columns) into shared memory, the "transform"
 // warps turn each block into an fp16 tile (exact for this format, see common.cuh) written straight
 // into the tensor core's 128-byte-swizzled K-major operand layout, and one thread issues
 // tcgen05.mma with that tile as A and a TMA tile of the expert's token rows as B, accumulating in
-// tensor memory.  Swap-AB: M = 128 weight rows, N = up to 256 tokens of one expert, so experts with
-// few tokens still fill the M dimension.  The dequantised weights exist only in shared memory.
+// tensor memory.  Swap-AB: M = 128 weight rows, N = up to kBN (256 or 128) tokens of one expert, so
+// experts with few tokens still fill the M dimension.  The dequantised weights exist only in
+// shared memory.
 //
 // Shaped by measurement on this part: every TMA operation costs an SM at least ~360 cycles
-// whatever its size, while big copies stream at ~90 B/clk.  So the weight blocks travel four
+// whatever its size, while big copies stream at ~90 B/clk.  So the weight blocks travel several
 // k-steps per copy, the token tile is a single box per k-step whose height (64/128/256 rows)
 // follows the tile's token count, and the three operand rings are sized separately (the token
 // ring's refill waits on L2, the A ring's only on the transform warps):
 //   weight ring  kWS stages x kWB blocks   (producer -> transform)
-//   token ring   kBS stages x 256 x 64     (producer -> MMA)
+//   token ring   kBS stages x kBN x 64     (producer -> MMA)
 //   A ring       kAS stages x 128 x 64     (transform -> MMA)
 // Barrier arrivals are one per warp.
 //
-//   gate/up kernel : per tile (expert, 128 interleaved gate/up rows, <=256 tokens), K = H.
+//   gate/up kernel : per tile (expert, 128 interleaved gate/up rows, <= kBN tokens), K = H.
 //                    B = the expert's bucketed fp16 token rows (the shared expert reads the fp16
 //                    activations directly: its rows are all tokens in order).  Epilogue:
 //                    act = silu(G) * U (G and U of one column i sit 16 TMEM lanes apart in the
 //                    same warp, paired with one shuffle), fp16, staged in shared memory and written
 //                    to the expert's act rows (only the tile's valid tokens).
-//   down kernel    : per tile (expert, 128 output rows, <=256 tokens), K = I.  B = act rows.
+//   down kernel    : per tile (expert, 128 output rows, <= kBN tokens), K = I.  B = act rows.
 //                    Epilogue: y * gate (routing gate, or sigmoid gate for the shared expert) added
 //                    into the token's fp32 accumulator row.  A warp's 32 x 32 block (32 output
 //                    rows = TMEM lanes, 32 tokens) is transposed through shared memory so that each
