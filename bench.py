@@ -359,6 +359,71 @@ def decode_gemv_only(shape, xs, reps, hbm, peak_src):
             "chain_kernels_us_eager": {k: round(v["avg_us"], 2) for k, v in prof.items()}}
 
 
+def small_batch_decode(shape, reps, hbm, peak_src):
+    """Decode batches of T = 1..16 tokens through both paths of the same 8 distinct layers: the
+    sparse GEMV path (a handle with decode_max_tokens = 16) and the grouped-GEMM prefill path (a
+    handle with decode_max_tokens = 0), each pass over the 8 layers replayed as one CUDA graph.
+    Per T: us per layer call for each path, the GEMV path's HBM fraction (algorithmic bytes = the
+    experts that receive a token + router + shared gate + x/out) and where the GEMM path wins."""
+    import torch
+    from bit_grouped_expert_router_b200 import _lib as M
+    from bit_grouped_expert_router_b200 import synth
+    n = 8
+    gemv, gemm, xs = [], [], []
+    for l in range(n):
+        w = synth.make_layer(shape, l, device="cuda")
+        gemv.append(M.Layer.from_shape(w, shape, max_tokens=16, decode_max_tokens=16))
+        gemm.append(M.Layer.from_shape(w, shape, max_tokens=16, decode_max_tokens=0))
+        del w
+        xs.append(synth.make_x(shape, l, 0, device="cuda", T=16))
+    expert_bytes = (shape.I // 64) * (shape.H // 64) * 4608 + (shape.H // 128) * (shape.I // 64) * 4608
+
+    def graph_us(layers, T):
+        outs = [torch.empty((T, shape.H), dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+
+        def step():
+            for l in range(n):
+                layers[l].forward(xs[l][:T], out=outs[l])
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            step()
+        torch.cuda.synchronize()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1000.0 / (reps * n)
+
+    rows, crossover = {}, None
+    for T in (1, 2, 4, 8, 16):
+        u_gemv, u_gemm = graph_us(gemv, T), graph_us(gemm, T)
+        active = statistics.mean(int(torch.unique(gemv[l].route(xs[l][:T])["idx"]).numel()) + 1
+                                 for l in range(n))
+        b = active * expert_bytes + shape.E * shape.H * 4 + shape.H * 4 + 2 * T * shape.H * 2
+        rows[str(T)] = {"gemv_us_per_layer": round(u_gemv, 2), "gemm_us_per_layer": round(u_gemm, 2),
+                        "gemv_us_per_token_layer": round(u_gemv / T, 2), "active_experts_mean": active,
+                        "gemv_hbm_frac": round(b / (u_gemv * 1e-6) / 1e9 / hbm, 4)}
+        if crossover is None and u_gemm < u_gemv:
+            crossover = T
+    for L in gemv + gemm:
+        assert L.status() == 0
+        L.close()
+    return {"layers": n, "timing": "CUDA graph of one pass over the layers, events", "per_T": rows,
+            "gemm_path_faster_from_T": crossover, "peak_source": f"{peak_src} hbm_gbs"}
+
+
 def run_configs(args, dist, peaks, peak_src):
     """The other prefill configurations' roofline fractions: prefill512 (HBM-bound: algorithmic
     bytes = weights of the experts that receive a token + router + shared gate + x/out, over the
@@ -458,11 +523,15 @@ def run_decode(args, dist, peaks, peak_src):
         L.close()
     del g
     gemv_only = decode_gemv_only(shape, xs, max(args.steps, 20), hbm, peak_src)
+    try:   # a measurement beside the decode line: must never cost the line itself
+        small = small_batch_decode(shape, max(args.steps, 20), hbm, peak_src)
+    except Exception as e:   # noqa: BLE001
+        small = {"error": f"{type(e).__name__}: {e}"[:300]}
     return {"metric": DECODE_METRIC,
             "value": round(us_layer, 3), "unit": "us/token/layer", "higher_is_better": False,
             "whole_layer_hbm_frac": round(layer_bytes / (us_layer * 1e-6) / 1e9 / hbm, 4),
             "whole_layer_bytes": layer_bytes, "roofline": roof, "kernels": prof,
-            "gemv_kernels_only": gemv_only,
+            "gemv_kernels_only": gemv_only, "small_batch": small,
             "gpu_launches_per_step": (1 if "decode_fused" in prof else 4) * n_layers}
 
 
