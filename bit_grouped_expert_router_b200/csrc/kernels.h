@@ -69,8 +69,8 @@ struct Ctx {
     int* hist;
     int* counts;
     int* offsets;
-    int4* tiles1;
-    int4* tiles2;
+    int4* tiles1;      // grouped-GEMM tile list {group, first bucket row, rows, 0}, ntiles[0] entries
+    int4* tiles2;      // the same list (both GEMMs walk one list; kept as a separate name)
     int* ntiles;
     int* perm;
     int* row_token;
