@@ -610,7 +610,9 @@ def run_reference(args, dist):
     w = synth.make_layer(shape, 0)
     x = synth.make_x(shape, 0, 0)
     ol = oracle.OracleLayer.from_shape(w, shape)
-    per_step = 8 if shape.T > 1 else 1
+    # 32 tokens per step for prefill, as cpu_baseline times them, so the oracle's OpenMP loop over
+    # tokens keeps every host core busy and the two CPU figures of one run agree
+    per_step = 32 if shape.T > 1 else 1
     t_tok = []
     for i in range(args.warmup + args.steps):
         tok = [(i * per_step + j) % shape.T for j in range(per_step)]

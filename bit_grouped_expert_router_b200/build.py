@@ -43,7 +43,21 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
+# The decode GEMVs feed 4-bit codes to fp32 FMAs as IEEE subnormals (code * 2^-149, see
+# csrc/decode.cu); those FMAs are written as explicit fma.rn.f32 in inline PTX so they keep
+# subnormals whatever the compiler flags say, and flush-to-zero builds are refused here as well so
+# no other arithmetic silently changes either.
+FORBIDDEN_FLAGS = ("-ftz=true", "--ftz=true", "--use_fast_math", "-use_fast_math")
+
+
+def check_flags(flags) -> None:
+    bad = [f for f in flags if f in FORBIDDEN_FLAGS]
+    if bad:
+        raise ValueError(f"libmoe must be built without flush-to-zero / fast math (got {bad})")
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+    check_flags(list(NVCC_FLAGS) + list(extra_flags))
     if not force and up_to_date():
         return LIB
     os.makedirs(BUILD, exist_ok=True)

@@ -155,7 +155,9 @@ int validate_config(const moe_config* c) {
         return fail(MOE_ERR_INVALID_ARG, "top_k must be in [1, min(num_experts, 32)]");
     if (c->has_shared != 0 && c->has_shared != 1) return fail(MOE_ERR_INVALID_ARG, "has_shared must be 0 or 1");
     if (c->max_tokens < 1 || c->max_tokens > 65536) return fail(MOE_ERR_INVALID_ARG, "max_tokens must be in [1, 65536]");
-    if (c->decode_max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "decode_max_tokens must be >= 0");
+    if (c->decode_max_tokens < 0 || c->decode_max_tokens > 65535)
+        return fail(MOE_ERR_INVALID_ARG,
+                    "decode_max_tokens must be in [0, 65535] (the GEMV path launches one grid slice per token)");
     if ((c->decode_max_tokens >= 2 || (c->flags & MOE_FLAG_DECODE_UNFUSED)) && c->top_k + c->has_shared > 16)
         return fail(MOE_ERR_INVALID_ARG, "the multi-kernel decode path supports top_k + has_shared <= 16");
     if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_DECODE_UNFUSED | MOE_FLAG_TEST_STALL))

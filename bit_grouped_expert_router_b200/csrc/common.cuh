@@ -55,6 +55,15 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
+// d = a * b + c in fp32, rounded once, with subnormal inputs and results kept: an explicit
+// fma.rn.f32 (no .ftz), so a build with -ftz=true or --use_fast_math cannot flush the subnormal
+// weight codes of the decode GEMVs to zero.  Not volatile: the compiler may schedule it freely.
+__device__ __forceinline__ float fma_keep_subnormal(float a, float b, float c) {
+    float d;
+    asm("fma.rn.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
     if (status) atomicOr(status, bit);
 }

@@ -9,7 +9,8 @@
 // Arithmetic per 64-column group c of a row:  sum_i W_i v_i = s * sum_i q_i v_i + b * sum_i v_i.
 // The code q_i becomes an fp32 operand in one byte-permute: a binary32 whose exponent field is
 // zero encodes mantissa * 2^-149, so a zero-extended nibble IS the value q * 2^-149 (an IEEE
-// subnormal, handled at full rate by FFMA without flush-to-zero).  The activations of the group
+// subnormal, handled at full rate by FFMA without flush-to-zero; the FMAs are explicit fma.rn.f32 so
+// no compiler flag can flush them).  The activations of the group
 // are pre-scaled by an exact power of two 2^K chosen from the group maximum so every product and
 // partial sum stays a normal number; the group result is rescaled by 2^(149-K).  Each byte of
 // (word & 0x0F0F0F0F) and ((word >> 4) & 0x0F0F0F0F) is one code, so the activations are stored
@@ -52,14 +53,14 @@ __device__ __forceinline__ float dot_group(const uint4& c0, const uint4& c1, con
         const uint32_t m1 = (w[i] >> 4) & 0x0F0F0F0Fu;
         const float4 x0 = *reinterpret_cast<const float4*>(vp + 8 * i);
         const float4 x1 = *reinterpret_cast<const float4*>(vp + 8 * i + 4);
-        a0 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4440)), x0.x, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4441)), x0.y, a1);
-        a0 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4442)), x0.z, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4443)), x0.w, a1);
-        a0 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4440)), x1.x, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4441)), x1.y, a1);
-        a0 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4442)), x1.z, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4443)), x1.w, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4440)), x0.x, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4441)), x0.y, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4442)), x0.z, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4443)), x0.w, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4440)), x1.x, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4441)), x1.y, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4442)), x1.z, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4443)), x1.w, a1);
     }
     return a0 + a1;
 }

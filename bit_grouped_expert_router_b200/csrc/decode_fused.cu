@@ -52,14 +52,14 @@ __device__ __forceinline__ float dot_group(const uint4& c0, const uint4& c1, con
         const uint32_t m1 = (w[i] >> 4) & 0x0F0F0F0Fu;
         const float4 x0 = *reinterpret_cast<const float4*>(vp + 8 * i);
         const float4 x1 = *reinterpret_cast<const float4*>(vp + 8 * i + 4);
-        a0 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4440)), x0.x, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4441)), x0.y, a1);
-        a0 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4442)), x0.z, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m0, 0u, 0x4443)), x0.w, a1);
-        a0 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4440)), x1.x, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4441)), x1.y, a1);
-        a0 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4442)), x1.z, a0);
-        a1 = fmaf(__uint_as_float(__byte_perm(m1, 0u, 0x4443)), x1.w, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4440)), x0.x, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4441)), x0.y, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4442)), x0.z, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4443)), x0.w, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4440)), x1.x, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4441)), x1.y, a1);
+        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4442)), x1.z, a0);
+        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4443)), x1.w, a1);
     }
     return a0 + a1;
 }

@@ -16,9 +16,16 @@
 // may return wrong results: serialise them.
 //
 // Set-up: the device address of the array is looked up (cudaGetSymbolAddress) the first time the
-// entry point runs on a device, with that device current.  That first call therefore makes a
-// runtime query that is not a stream operation; make it before starting any stream capture.
+// entry point runs in a CUDA context, with that context current.  That first call therefore makes
+// a runtime query that is not a stream operation; make it before starting any stream capture.
+// The address is cached per context (keyed on the driver's unique context id, not on the device
+// ordinal): after cudaDeviceReset, or after the primary context is released and created again,
+// the module is loaded anew and the array may sit at another address, so the first call in the
+// new context looks it up again -- that call, too, belongs outside any capture.
+#include <cudaTypedefs.h>
+
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -111,8 +118,33 @@ __global__ void __launch_bounds__(256) route_static_topk(const float* __restrict
 }
 
 std::mutex g_static_mu;
-constexpr int kMaxDevices = 128;
-void* g_static_ptr[kMaxDevices] = {};
+std::unordered_map<unsigned long long, void*> g_static_ptr;   // context id -> array address
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (0 if none is current yet).
+bool current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return false;
+    *id = 0;
+    return ctx == nullptr || get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 int static_fail(int code, const char* msg) {
     set_last_error(msg);  // reported by moe_last_error() on this thread
@@ -135,18 +167,26 @@ extern "C" int moe_route_static(const uint16_t* x, int32_t T, int32_t H, const f
         return static_fail(MOE_ERR_TOO_LARGE,
                            "moe_route_static: T * (H/32) * E exceeds the static scratch (MOE_ROUTE_STATIC_SCRATCH_FLOATS)");
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return static_fail(MOE_ERR_CUDA, "moe_route_static: no current CUDA device");
+    if (cudaGetDevice(&dev) != cudaSuccess) return static_fail(MOE_ERR_CUDA, "moe_route_static: no current CUDA device");
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_static_mu);
-        if (!g_static_ptr[dev]) {
+        unsigned long long ctx = 0;
+        if (!current_context_id(&ctx)) return static_fail(MOE_ERR_CUDA, "moe_route_static: cannot identify the CUDA context");
+        auto it = ctx ? g_static_ptr.find(ctx) : g_static_ptr.end();
+        if (it != g_static_ptr.end()) {
+            scratch = it->second;
+        } else {
+            // first call in this context (cudaGetSymbolAddress also makes the device's primary
+            // context current when none is): look the array up, then key it on the context id
             void* p = nullptr;
             const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
             if (e != cudaSuccess || !p) return static_fail(MOE_ERR_CUDA, "moe_route_static: cudaGetSymbolAddress failed");
-            g_static_ptr[dev] = p;
+            if (!current_context_id(&ctx) || ctx == 0)
+                return static_fail(MOE_ERR_CUDA, "moe_route_static: no CUDA context after set-up");
+            g_static_ptr[ctx] = p;
+            scratch = p;
         }
-        scratch = g_static_ptr[dev];
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* part = static_cast<float*>(scratch);

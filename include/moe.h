@@ -90,7 +90,8 @@ typedef struct {
     int32_t has_shared;        /* 1: one always-on shared expert with a sigmoid gate */
     int32_t max_tokens;        /* largest T that moe_forward / moe_route accept */
     int32_t decode_max_tokens; /* T <= this runs the sparse-GEMV decode path; larger T runs the
-                                  bucketed grouped-GEMM prefill path.  0 = always prefill path.
+                                  bucketed grouped-GEMM prefill path.  0 = always prefill path;
+                                  at most 65535.
                                   With decode_max_tokens >= 2 (or MOE_FLAG_DECODE_UNFUSED) the
                                   multi-kernel GEMV path needs top_k + has_shared <= 16. */
     uint32_t flags;            /* MOE_FLAG_* */
@@ -112,7 +113,9 @@ typedef struct {
     const float *shared_gate;
 } moe_weights;
 
-/* Create a layer on `device`: validate cfg, check the device is sm_100, allocate the handle's
+/* Source: the layer interface this library exposes (create a layer, then run it on [T, H] bf16
+ * activations on a stream); the pages describe the engine, not a layer-level call.
+ * Create a layer on `device`: validate cfg, check the device is sm_100, allocate the handle's
  * workspace (sized for cfg->max_tokens) and repack the weights into the handle's own kernel
  * layout with kernels enqueued on `stream`.  moe_create synchronises `stream` before returning,
  * so the caller may free its weight buffers as soon as it returns.  On success *out receives the
@@ -122,18 +125,24 @@ typedef struct {
 MOE_API int moe_create(const moe_config *cfg, const moe_weights *w, int device, void *stream,
                moe_handle **out);
 
-/* out[T, H] (bf16) = the layer applied to x[T, H] (bf16), both device pointers.  T == 0 is a
+/* Source: the forward pass of the layer as defined at the top of this file; prefill runs the
+ * bucketed grouped GEMM with in-GEMM 4-bit reconstruction and decode the sparse GEMV over the
+ * selected experts ("Perplexity Open-Sources Lily...", section "The optimizations follow the
+ * workload"; "A Rust + Metal Inference Engine..." body).
+ * out[T, H] (bf16) = the layer applied to x[T, H] (bf16), both device pointers.  T == 0 is a
  * no-op returning MOE_OK.  Errors: INVALID_ARG (null/misaligned pointer, T < 0), TOO_LARGE
  * (T > max_tokens), CUDA (launch failure).  Device-side errors surface via moe_status(). */
 MOE_API int moe_forward(moe_handle *h, const uint16_t *x, int32_t T, uint16_t *out, void *stream);
 
-/* The same with HOST buffers: copies x to the device, runs moe_forward, copies out back and
+/* Source: library convenience (no passage): the forward pass with host buffers.
+ * The same with HOST buffers: copies x to the device, runs moe_forward, copies out back and
  * synchronises `stream` before returning (so the host buffer is ready).  Pinned host memory is
  * fastest; pageable memory works.  Uses handle-owned device staging buffers (no allocation). */
 MOE_API int moe_forward_host(moe_handle *h, const uint16_t *x_host, int32_t T, uint16_t *out_host,
                      void *stream);
 
-/* moe_forward_host without the final synchronisation: the copy in, the layer and the copy out are
+/* Source: library convenience (no passage).
+ * moe_forward_host without the final synchronisation: the copy in, the layer and the copy out are
  * enqueued on `stream` and the call returns.  x_host must stay unchanged and out_host unread until
  * the stream has passed the copy out (synchronise the stream or an event recorded after the call).
  * With pinned host memory the copies are asynchronous, so calls on different handles issued to
@@ -144,7 +153,9 @@ MOE_API int moe_forward_host(moe_handle *h, const uint16_t *x_host, int32_t T, u
 MOE_API int moe_forward_host_async(moe_handle *h, const uint16_t *x_host, int32_t T, uint16_t *out_host,
                            void *stream);
 
-/* Routing and bucketing only (the first steps of the prefill path), with their results copied
+/* Source: "Perplexity Open-Sources Lily...", section "The optimizations follow the workload":
+ * expert routing is kept on the GPU with no CPU synchronisation; this call exposes its results.
+ * Routing and bucketing only (the first steps of the prefill path), with their results copied
  * to caller device buffers (any output pointer may be NULL to skip it):
  *   idx[T, k] int32      experts per token, descending logit
  *   gates[T, k] fp32     renormalised softmax gates, same order
@@ -157,12 +168,14 @@ MOE_API int moe_forward_host_async(moe_handle *h, const uint16_t *x_host, int32_
 MOE_API int moe_route(moe_handle *h, const uint16_t *x, int32_t T, int32_t *idx, float *gates,
               float *shared_gate, int32_t *offsets, int32_t *perm, void *stream);
 
-/* Synchronise the stream of the handle's last call, read and clear the device status word.
+/* Source: library convenience (no passage).
+ * Synchronise the stream of the handle's last call, read and clear the device status word.
  * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS, MOE_ERR_RANGE (the most severe
  * recorded, in that order of precedence reversed: timeout > bounds > range) or MOE_ERR_CUDA. */
 MOE_API int moe_status(moe_handle *h);
 
-/* Debug: copy `bytes` of an internal workspace buffer to a caller device buffer (stream-ordered).
+/* Source: library convenience (no passage).
+ * Debug: copy `bytes` of an internal workspace buffer to a caller device buffer (stream-ordered).
  * which: 0 = expert activations act[rows, I] (fp16, bucket order, prefill path),
  *        1 = fp16 copy of the activations x16[T, H] (prefill path),
  *        2 = router logits [T, E] (fp32, tensor-core router only),
@@ -170,7 +183,8 @@ MOE_API int moe_status(moe_handle *h);
  * Errors: INVALID_ARG when `which` is unknown or `bytes` exceeds the buffer. */
 MOE_API int moe_debug_copy(moe_handle *h, int which, void *dst, size_t bytes, void *stream);
 
-/* Per-kernel timing.  While enabled, moe_forward records a CUDA event on the call's stream before
+/* Source: library convenience (no passage).
+ * Per-kernel timing.  While enabled, moe_forward records a CUDA event on the call's stream before
  * its first kernel and after each kernel it launches (events are created by moe_profile_enable;
  * up to 1024 calls are recorded, later calls run unrecorded).  Do not enable it while capturing a
  * CUDA graph.  moe_profile_read synchronises those events, writes per kernel slot the summed
@@ -184,13 +198,16 @@ MOE_API int moe_debug_copy(moe_handle *h, int which, void *dst, size_t bytes, vo
 MOE_API int moe_profile_enable(moe_handle *h, int enable);
 MOE_API int moe_profile_read(moe_handle *h, float *ms, int32_t *launches);
 
-/* Bytes of device memory a handle with this configuration owns (repacked weights + workspace). */
+/* Source: library convenience (no passage).
+ * Bytes of device memory a handle with this configuration owns (repacked weights + workspace). */
 MOE_API size_t moe_device_bytes(const moe_config *cfg);
 
-/* Message describing the last error returned on the calling thread ("" if none). */
+/* Source: library convenience (no passage).
+ * Message describing the last error returned on the calling thread ("" if none). */
 MOE_API const char *moe_last_error(void);
 
-/* Free the handle and all device memory it owns.  Synchronises the device first.  NULL is a no-op. */
+/* Source: library convenience (no passage).
+ * Free the handle and all device memory it owns.  Synchronises the device first.  NULL is a no-op. */
 MOE_API void moe_destroy(moe_handle *h);
 
 /* Routing for callers that cannot allocate device memory.  No counterpart on the pages: this is a
@@ -200,21 +217,30 @@ MOE_API void moe_destroy(moe_handle *h);
  * create a moe_handle.  This entry point computes, for x[T, H] (bf16, device), the router's top-k
  * experts idx[T, k] (int32, device) and their renormalised gates gates[T, k] (fp32, device) from
  * the caller's router[E, H] (fp32, device, public layout) and optional router_bias[E] (fp32 or
- * NULL), exactly as moe_route does, on the current device and `stream`.  It allocates nothing:
+ * NULL), with the same selection rule as moe_route (descending logit, ties to the lower index,
+ * softmax renormalised over the selection), on the current device and `stream`.  The logits are
+ * fp32 sums taken in 32-column slices on CUDA cores, a different summation order from
+ * moe_route's tensor-core router at prefill sizes, so idx agrees with moe_route (and with the
+ * exact result) whenever adjacent top-(k+1) logits are further apart than fp32 rounding, and the
+ * gates agree to about 1e-6.  It allocates nothing:
  * its only scratch (split-K partial logits, T * (H/32) * E floats) lives in a fixed array of
  * MOE_ROUTE_STATIC_SCRATCH_FLOATS floats (1 MiB) compiled into the library, which every GPU that
  * loads the library holds until the process exits.  Larger requests return MOE_ERR_TOO_LARGE.
  * The array is shared by all calls and keeps the last call's contents (each call overwrites what
  * it reads, so nothing needs clearing); calls that overlap on the GPU race on it -- serialise
- * them.  The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make that first call before any stream capture begins.
+ * them.  The first call in a CUDA context looks up the array's device address
+ * (cudaGetSymbolAddress) with that context current and caches it per context; make that first
+ * call before any stream capture begins.  After cudaDeviceReset (or once the primary context has
+ * been released and created again) the next call looks the address up again, so it too must be
+ * made outside a capture.
  * Errors: INVALID_ARG (H % 32 != 0, k or E out of range, NULL pointer), TOO_LARGE, CUDA. */
 #define MOE_ROUTE_STATIC_SCRATCH_FLOATS 262144
 MOE_API int moe_route_static(const uint16_t *x, int32_t T, int32_t H, const float *router,
                              const float *router_bias, int32_t E, int32_t k, int32_t *idx,
                              float *gates, void *stream);
 
-/* Library version as major*10000 + minor*100 + patch. */
+/* Source: library convenience (no passage).
+ * Library version as major*10000 + minor*100 + patch. */
 MOE_API int moe_version(void);
 
 #ifdef __cplusplus

@@ -45,7 +45,7 @@ def test_device_bytes_counts_the_repacked_layer(lib):
 
 @pytest.mark.parametrize("bad", [dict(group=32), dict(H=200), dict(I=96), dict(E=0), dict(E=300),
                                  dict(k=0), dict(k=33, E=64), dict(k=9, E=8), dict(max_tokens=0),
-                                 dict(decode_max_tokens=-1), dict(flags=0x8),
+                                 dict(decode_max_tokens=-1), dict(decode_max_tokens=65536), dict(flags=0x8),
                                  dict(k=16, decode_max_tokens=2)])
 def test_invalid_config_is_rejected_before_any_cuda_call(lib, bad):
     cfg = _cfg(**bad)
@@ -83,3 +83,26 @@ def test_create_without_a_gpu_reports_cuda_error(lib):
     rc = lib.moe_create(ctypes.byref(_cfg()), ctypes.byref(w), 0, None, ctypes.byref(h))
     assert rc in (M.MOE_ERR_CUDA, M.MOE_ERR_INVALID_ARG)
     assert lib.moe_last_error().decode()
+
+
+def test_flush_to_zero_builds_are_refused():
+    """The decode GEMVs carry 4-bit codes as fp32 subnormals; the build refuses flush-to-zero and
+    fast-math flags, and its own flag list holds none of them."""
+    for f in B.FORBIDDEN_FLAGS:
+        assert f not in B.NVCC_FLAGS
+        with pytest.raises(ValueError):
+            B.check_flags(list(B.NVCC_FLAGS) + [f])
+    B.check_flags(B.NVCC_FLAGS)
+
+
+def test_subnormal_fmas_are_explicit_ptx():
+    """Every FMA that multiplies a subnormal weight code is the explicit fma.rn.f32 helper, never
+    fmaf (which -ftz=true would turn into a flushing instruction)."""
+    import os
+    import re
+    csrc = os.path.join(os.path.dirname(B.__file__), "csrc")
+    for name in os.listdir(csrc):
+        if not name.endswith(".cu"):
+            continue
+        src = open(os.path.join(csrc, name)).read()
+        assert not re.search(r"fmaf\(__uint_as_float\(__byte_perm", src), name

@@ -277,6 +277,18 @@ def test_sparse_equals_dense_with_zeroed_gates(shape):
     assert np.linalg.norm(ys - yd) <= 1e-12 * np.linalg.norm(yd)
 
 
+def test_sparse_equals_dense_at_the_full_layer_shapes():
+    """The same check at the full layer shapes (H = 2048, E = 256, k = 8, I = 512, shared
+    expert): a few tokens through all 256 experts with the unselected gates zeroed."""
+    shape = synth.Shape("full_dense", T=3, H=2048, E=256, k=8, I=512, seed=1)
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    ys = ol.forward(x)
+    yd = ol.forward(x, dense=True)
+    assert np.linalg.norm(ys - yd) <= 1e-12 * np.linalg.norm(yd)
+
+
 def test_token_subset_matches_full_run():
     shape = TINY
     w = synth.make_layer(shape)
