@@ -485,15 +485,20 @@ def run_decode(args, dist, peaks, peak_src):
         for l in range(n_layers):
             layers[l].forward(xs[l], out=outs[l])
 
-    eager()
-    torch.cuda.synchronize()
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
+    def graph_ms():
         eager()
-    torch.cuda.synchronize()
-    ms = timed(g.replay, max(args.steps, 20) * 5, args.warmup, dist)
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            eager()
+        torch.cuda.synchronize()
+        t = timed(g.replay, max(args.steps, 20) * 5, args.warmup, dist)
+        del g
+        return t
+
+    ms = graph_ms()
     us_layer = ms * 1000.0 / n_layers
     prof = profile_pass(layers, eager, max(args.steps, 20))
     expert_bytes = (shape.I // 64) * (shape.H // 64) * 4608 + (shape.H // 128) * (shape.I // 64) * 4608
@@ -521,7 +526,6 @@ def run_decode(args, dist, peaks, peak_src):
     for L in layers:
         assert L.status() == 0
         L.close()
-    del g
     gemv_only = decode_gemv_only(shape, xs, max(args.steps, 20), hbm, peak_src)
     try:   # a measurement beside the decode line: must never cost the line itself
         small = small_batch_decode(shape, max(args.steps, 20), hbm, peak_src)

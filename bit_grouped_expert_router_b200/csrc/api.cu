@@ -9,6 +9,7 @@
 // Decode path (T <= decode_max_tokens): split-K router -> top-k/gates -> sparse GEMV gate/up +
 //   SwiGLU -> sparse GEMV down + gated combine (bf16 out).
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstdarg>
@@ -16,6 +17,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -43,6 +45,18 @@ int fail(int code, const char* fmt, ...) {
         if (_e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(_e)); \
     } while (0)
 
+// NVTX range around one launch (or one entry-point call) so a timeline tool attributes device
+// time to the library's phases; header-only NVTX, a no-op when no tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+#define MOE_LAUNCH(name, expr)    \
+    do {                          \
+        NvtxRange _nvtx(name);    \
+        CUDA_TRY(expr);           \
+    } while (0)
+
 struct DeviceGuard {
     int prev = -1;
     bool changed = false;
@@ -67,8 +81,8 @@ struct Layout {
     size_t o_wrt, o_rbias, o_sgw, o_router32;   // offsets inside the router region
     // workspace offsets
     size_t o_part, o_idx, o_gates, o_sg, o_hist, o_counts, o_offsets, o_tiles, o_ntiles, o_perm, o_rtok,
-        o_rgate, o_x16, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_counters, o_stage_x, o_stage_out, o_dfz_rpart,
-        o_dfz_gu, o_dfz_outacc, o_dfz_cnt, o_dfz_bar, ws_bytes;
+        o_rgate, o_x16, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_stage_x, o_stage_out, o_dfz_ticket,
+        o_dfz_slots, o_dfz_outacc, o_dfz_cnt, o_dfz_dirty, ws_bytes;
 };
 
 struct Layout;
@@ -130,14 +144,13 @@ Layout make_layout(const moe_config& c) {
     L.o_dact = take(sizeof(float) * (size_t)std::max(L.Tdec, 1) * (L.k + 1) * L.I);
     L.o_dscale = take(sizeof(float) * 2 * (size_t)std::max(L.Tdec, 1) * (L.k + 1) * (L.I / 64));
     L.o_status = take(sizeof(uint32_t) * 4);
-    L.o_counters = take(sizeof(unsigned) * 64);
     L.o_stage_x = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
     L.o_stage_out = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
-    L.o_dfz_rpart = take(sizeof(float) * 4 * (size_t)L.E);
-    L.o_dfz_gu = take(sizeof(float) * (size_t)(L.k + 1) * 4 * 2 * L.I);
+    L.o_dfz_ticket = take(sizeof(unsigned long long));
+    L.o_dfz_slots = take(sizeof(unsigned long long) * (size_t)L.E);
     L.o_dfz_outacc = take(sizeof(float) * (size_t)L.H);
-    L.o_dfz_cnt = take(sizeof(unsigned) * (size_t)(L.H / 32));
-    L.o_dfz_bar = take(sizeof(unsigned long long) * 16 * 32);
+    L.o_dfz_cnt = take(sizeof(unsigned) * (size_t)(L.H / 128));
+    L.o_dfz_dirty = take(sizeof(unsigned));
     L.ws_bytes = o;
     return L;
 }
@@ -160,7 +173,8 @@ int validate_config(const moe_config* c) {
                     "decode_max_tokens must be in [0, 65535] (the GEMV path launches one grid slice per token)");
     if ((c->decode_max_tokens >= 2 || (c->flags & MOE_FLAG_DECODE_UNFUSED)) && c->top_k + c->has_shared > 16)
         return fail(MOE_ERR_INVALID_ARG, "the multi-kernel decode path supports top_k + has_shared <= 16");
-    if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_DECODE_UNFUSED | MOE_FLAG_TEST_STALL))
+    if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_DECODE_UNFUSED | MOE_FLAG_POISON_WORKSPACE |
+                               MOE_FLAG_TEST_STALL))
         return fail(MOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
     return MOE_OK;
 }
@@ -224,6 +238,9 @@ struct moe_handle {
     uint16_t* wsplit = nullptr;
     cudaStream_t last_stream = nullptr;
     bool inexact_scales = false;
+    // batch-1 decode: the fused kernel's geometry, when the shape and the device allow it
+    bool fused_ok = false;
+    DecodeGeom dgeom{};
 };
 
 namespace {
@@ -251,10 +268,9 @@ int check_call(moe_handle* h, const void* x, int32_t T, const void* out, bool ne
 
 bool use_decode(const moe_handle* h, int T) { return T <= h->cfg.decode_max_tokens; }
 
-// The single-kernel decode handles T == 1 when its per-warp k-ranges fit (H <= 2048, I <= 2048).
-bool fused_decode_ok(const moe_handle* h) {
-    return !(h->cfg.flags & MOE_FLAG_DECODE_UNFUSED) && h->L.H / 64 <= 8 * 4 && h->L.I / 64 <= 8 * 4;
-}
+// The fused kernel serves T == 1 when the shape fits its geometry and all of its clusters can be
+// resident at once (decided at create); otherwise the multi-kernel GEMV chain does.
+bool fused_decode_ok(const moe_handle* h) { return h->fused_ok && !(h->cfg.flags & MOE_FLAG_DECODE_UNFUSED); }
 
 // Profiling: one event before the first kernel of a call and one after each kernel.
 struct Prof {
@@ -280,20 +296,20 @@ struct Prof {
 
 int enqueue_routing(moe_handle* h, Prof& pf, const Ctx& c, bool decode, cudaStream_t st) {
     if (decode || (h->cfg.flags & MOE_FLAG_ROUTER_SIMT)) {
-        CUDA_TRY(launch_router_simt(c, st));
+        MOE_LAUNCH("moe.router_simt", launch_router_simt(c, st));
     } else {
         CUtensorMap tm_x;
         const int rc = encode_rows_map(&tm_x, c.x, c.T, c.H, 128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
         if (rc != MOE_OK) return rc;
-        CUDA_TRY(launch_router_tc(c, h->tm_wsplit, tm_x, router_n_exp(h->L), st));
+        MOE_LAUNCH("moe.router_tc", launch_router_tc(c, h->tm_wsplit, tm_x, router_n_exp(h->L), st));
     }
     pf.mark(0);
-    CUDA_TRY(launch_topk(c, !decode, st));
+    MOE_LAUNCH("moe.topk", launch_topk(c, !decode, st));
     pf.mark(1);
     if (!decode) {
-        CUDA_TRY(launch_bucket_scan(c, st));
+        MOE_LAUNCH("moe.bucket_scan", launch_bucket_scan(c, st));
         pf.mark(2);
-        CUDA_TRY(launch_scatter(c, st));
+        MOE_LAUNCH("moe.scatter", launch_scatter(c, st));
         pf.mark(3);
     }
     return MOE_OK;
@@ -359,7 +375,20 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMalloc(weights %zu B): %s", L.weights_bytes, cudaGetErrorString(e)));
     e = cudaMalloc(&h->ws, L.ws_bytes);
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMalloc(workspace %zu B): %s", L.ws_bytes, cudaGetErrorString(e)));
-    e = cudaMemsetAsync(h->ws, 0, L.ws_bytes, st);
+    if (cfg->flags & MOE_FLAG_POISON_WORKSPACE) {
+        // 0xFF bytes everywhere (NaN floats, -1 indices), then zero only the words the kernels
+        // count on starting at zero: the bucketing histograms, the status words and the fused
+        // decode's call ticket and router words; its dirty word is raised, so the first decode
+        // call resets its accumulator and counters on the device
+        e = cudaMemsetAsync(h->ws, 0xFF, L.ws_bytes, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_hist, 0, sizeof(int) * (size_t)L.nblk_max * L.E, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_status, 0, sizeof(uint32_t) * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_ticket, 0, sizeof(unsigned long long), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_slots, 0, sizeof(unsigned long long) * (size_t)L.E, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_dirty, 0x01, sizeof(unsigned), st);
+    } else {
+        e = cudaMemsetAsync(h->ws, 0, L.ws_bytes, st);
+    }
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e)));
 
     uint8_t* w_gu = h->wbuf;
@@ -442,15 +471,22 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.dact = reinterpret_cast<float*>(ws + L.o_dact);
     c.dscale = reinterpret_cast<float*>(ws + L.o_dscale);
     c.status = status;
-    c.counters = reinterpret_cast<unsigned*>(ws + L.o_counters);
-    c.dfz.rpart = reinterpret_cast<float*>(ws + L.o_dfz_rpart);
-    c.dfz.gu = reinterpret_cast<float*>(ws + L.o_dfz_gu);
+    c.dfz.ticket = reinterpret_cast<unsigned long long*>(ws + L.o_dfz_ticket);
+    c.dfz.slots = reinterpret_cast<unsigned long long*>(ws + L.o_dfz_slots);
     c.dfz.outacc = reinterpret_cast<float*>(ws + L.o_dfz_outacc);
     c.dfz.cnt = reinterpret_cast<unsigned*>(ws + L.o_dfz_cnt);
-    c.dfz.bar = reinterpret_cast<unsigned long long*>(ws + L.o_dfz_bar);
+    c.dfz.dirty = reinterpret_cast<unsigned*>(ws + L.o_dfz_dirty);
+
+    if (decode_fused_geometry(L.H, L.I, L.E, L.k, cfg->has_shared, &h->dgeom)) {
+        int nclusters = 0;
+        e = decode_fused_prepare(h->dgeom);
+        if (e == cudaSuccess) e = decode_fused_max_clusters(h->dgeom, &nclusters);
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "decode kernel set-up: %s", cudaGetErrorString(e)));
+        h->fused_ok = nclusters >= h->dgeom.units;
+    }
 
     for (int hs = 0; hs < 3 && rc == MOE_OK; ++hs) {
-        const int box = 64 << hs;   // token tile box: 64, 128 or 256 rows
+        const int box = token_box_rows(hs);   // token tile box: 64, 128 or 256 rows
         rc = encode_rows_map(&h->maps_gu.m[0][hs], c.xp, L.Tm * L.k, L.H, box);
         if (rc == MOE_OK) rc = encode_rows_map(&h->maps_gu.m[1][hs], c.x16, L.Tm, L.H, box);
         if (rc == MOE_OK) rc = encode_rows_map(&h->maps_dn.m[0][hs], c.act, L.rows_cap, L.I, box);
@@ -467,6 +503,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
 int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void* stream) {
     int rc = check_call(h, x, T, out, true);
     if (rc != MOE_OK || T == 0) return rc;
+    NvtxRange range("moe_forward");
     DeviceGuard guard(h->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;
@@ -474,25 +511,25 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     const Ctx c = make_ctx(h, T, x, out, decode);
     Prof pf(h, st);
     if (decode && T == 1 && fused_decode_ok(h)) {
-        CUDA_TRY(launch_decode_fused(c, h->num_sms, st));
+        MOE_LAUNCH("moe.decode_fused", launch_decode_fused(c, h->dgeom, st));
         pf.mark(9);
         return MOE_OK;
     }
     rc = enqueue_routing(h, pf, c, decode, st);
     if (rc != MOE_OK) return rc;
     if (decode) {
-        CUDA_TRY(launch_gemv_gateup(c, st));
+        MOE_LAUNCH("moe.gemv_gateup", launch_gemv_gateup(c, st));
         pf.mark(7);
-        CUDA_TRY(launch_gemv_down(c, st));
+        MOE_LAUNCH("moe.gemv_down", launch_gemv_down(c, st));
         pf.mark(8);
     } else {
-        CUDA_TRY(launch_gather_rows(c, h->num_sms, st));
+        MOE_LAUNCH("moe.gather_rows", launch_gather_rows(c, h->num_sms, st));
         pf.mark(10);
-        CUDA_TRY(launch_gemm_gateup(c, h->maps_gu, h->num_sms, st));
+        MOE_LAUNCH("moe.gemm_gateup", launch_gemm_gateup(c, h->maps_gu, h->num_sms, st));
         pf.mark(4);
-        CUDA_TRY(launch_gemm_down(c, h->maps_dn, h->num_sms, st));
+        MOE_LAUNCH("moe.gemm_down", launch_gemm_down(c, h->maps_dn, h->num_sms, st));
         pf.mark(5);
-        CUDA_TRY(launch_finalize(c, st));
+        MOE_LAUNCH("moe.finalize", launch_finalize(c, st));
         pf.mark(6);
     }
     return MOE_OK;
@@ -540,9 +577,9 @@ int moe_route(moe_handle* h, const uint16_t* x, int32_t T, int32_t* idx, float* 
     rc = enqueue_routing(h, pf, c, decode, st);
     if (rc != MOE_OK) return rc;
     if (decode) {
-        CUDA_TRY(launch_topk(c, true, st));
-        CUDA_TRY(launch_bucket_scan(c, st));
-        CUDA_TRY(launch_scatter(c, st));
+        MOE_LAUNCH("moe.topk", launch_topk(c, true, st));
+        MOE_LAUNCH("moe.bucket_scan", launch_bucket_scan(c, st));
+        MOE_LAUNCH("moe.scatter", launch_scatter(c, st));
     }
     const Layout& L = h->L;
     if (idx) CUDA_TRY(cudaMemcpyAsync(idx, c.idx, sizeof(int) * (size_t)T * L.k, cudaMemcpyDeviceToDevice, st));
@@ -560,13 +597,9 @@ int moe_status(moe_handle* h) {
     uint32_t s = 0;
     CUDA_TRY(cudaMemcpy(&s, h->base.status, sizeof s, cudaMemcpyDeviceToHost));
     CUDA_TRY(cudaMemset(h->base.status, 0, sizeof s));
-    if (s & MOE_STATUS_TIMEOUT) {
-        // a kernel gave up part-way: put the fused decode's self-cleaning state back to zero
-        CUDA_TRY(cudaMemset(h->base.dfz.bar, 0, sizeof(unsigned long long) * 16 * 32));
-        CUDA_TRY(cudaMemset(h->base.dfz.cnt, 0, sizeof(unsigned) * (size_t)(h->L.H / 32)));
-        CUDA_TRY(cudaMemset(h->base.dfz.outacc, 0, sizeof(float) * (size_t)h->L.H));
-        return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
-    }
+    // (a fused decode call that gave up part-way has raised the workspace's dirty word; the next
+    // such call resets its state on the device, so nothing needs resetting here)
+    if (s & MOE_STATUS_TIMEOUT) return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
     if (s & MOE_STATUS_BOUNDS) return fail(MOE_ERR_DEVICE_BOUNDS, "a device-side index check failed");
     if (s & MOE_STATUS_RANGE) return fail(MOE_ERR_RANGE, "a value exceeded the fp16 operand range");
     return MOE_OK;

@@ -13,6 +13,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libmoe targets sm_100a (B200) only"
 #endif
@@ -62,6 +64,17 @@ __device__ __forceinline__ float fma_keep_subnormal(float a, float b, float c) {
     float d;
     asm("fma.rn.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
+}
+
+// Programmatic dependent launch.  Every kernel of the forward path is launched as a programmatic
+// dependent of the previous kernel in its stream (launch_pdl), so its CTAs may start while that
+// kernel drains.  griddep_wait() blocks until the previous grid has completed and its memory is
+// visible; every such kernel calls it first, in every CTA, before reading anything (that keeps the
+// chain transitive: a grid completes only after its predecessor has).  It is a no-op in a grid
+// launched the ordinary way.  griddep_launch_dependents() lets the next grid be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
@@ -330,6 +343,23 @@ __device__ __forceinline__ __half2 codes_to_half2(uint32_t word, int s) {
     uint32_t v = ((word >> (4 * s)) & 0x000F000Fu) | 0x64006400u;
     __half2 h = *reinterpret_cast<__half2*>(&v);
     return __hsub2(h, __half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+}
+
+// Host: launch `kernel` as a programmatic dependent of the previous kernel in `st`.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

@@ -113,6 +113,8 @@ __device__ __forceinline__ float row_dot(const uint8_t* wb, int row, int c0, int
 constexpr int kGateupThreads = 512;
 
 __global__ void __launch_bounds__(kGateupThreads) gemv_gateup_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ __align__(16) float sm[];
     const int mt = blockIdx.x, j = blockIdx.y, t = blockIdx.z;
     const int nslot = c.k + c.has_shared;
@@ -190,6 +192,8 @@ __global__ void __launch_bounds__(kGateupThreads) gemv_gateup_kernel(Ctx c) {
 }
 
 __global__ void __launch_bounds__(1024) gemv_down_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ __align__(16) float sm[];
     const int hc = blockIdx.x, t = blockIdx.y;
     const int nslot = c.k + c.has_shared;
@@ -235,8 +239,7 @@ cudaError_t launch_gemv_gateup(const Ctx& c, cudaStream_t st) {
     const int KS = c.H / 64;
     const size_t smem = sizeof(float) * ((size_t)c.H + 2 * KS + 512 + 4);
     dim3 grid(c.I / 64, c.k + 1, c.T);
-    gemv_gateup_kernel<<<grid, kGateupThreads, smem, st>>>(c);
-    return cudaGetLastError();
+    return launch_pdl(gemv_gateup_kernel, grid, dim3(kGateupThreads), smem, st, c);
 }
 
 cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st) {
@@ -245,8 +248,7 @@ cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st) {
     if (threads > 1024) return cudaErrorInvalidConfiguration;   // k + shared > 16 slots
     const size_t smem = sizeof(float) * ((size_t)nslot * c.I + (size_t)threads);
     dim3 grid(c.H / 32, c.T);
-    gemv_down_kernel<<<grid, threads, smem, st>>>(c);
-    return cudaGetLastError();
+    return launch_pdl(gemv_down_kernel, grid, dim3(threads), smem, st, c);
 }
 
 }  // namespace moe

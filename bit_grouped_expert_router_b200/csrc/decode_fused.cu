@@ -1,29 +1,46 @@
-// decode_fused.cu -- batch-1 decode of one MoE layer in a single cooperative kernel.
+// decode_fused.cu -- batch-1 decode of one MoE layer in a single kernel of CTA pairs.
 //
-// A decode token moves ~18 MB (router 2 MiB + 9 experts x 1.69 MiB), about 2.8 us of HBM time, so
-// launch gaps and the first-byte latency of each dependent step dominate a multi-kernel chain.
-// Following the pages' decode levers -- fuse the kernel chain and run independent work
-// concurrently ("A Rust + Metal Inference Engine..." body; "Perplexity Open-Sources Lily..."
-// section "Generation has a different bottleneck") -- one persistent grid (one 512-thread CTA
-// per SM, co-resident by cooperative launch) runs three phases separated by two grid barriers:
+// A decode token moves ~18 MB (router 2 MiB + 9 experts x 1.69 MiB): about 2.8 us of HBM time,
+// so what decides the layer's time is how many dependent memory round trips lie on its critical
+// path and how much of the weight stream is in flight at once.  The pages' decode levers are to
+// fuse the kernel chain and to run independent work concurrently ("A Rust + Metal Inference
+// Engine..." body; "Perplexity Open-Sources Lily..." section "Generation has a different
+// bottleneck").  Here the whole layer is one grid of 2-CTA clusters, one cluster per work unit
+// (expert slot j, 64-column slice mt of the intermediate dimension):
 //
-//   phase 0  router logits (E x 4 quarter-row dot products, fp32) and, concurrently, the shared
-//            expert's gate/up GEMV (it needs no routing); every CTA also stages the token.
-//   phase 1  every CTA reduces the logits and picks the top k (identical result everywhere), then
-//            the k routed experts' gate/up GEMVs.
-//   phase 2  down GEMVs: a CTA owns one expert slot, builds act = silu(G) * U for it, streams the
-//            down blocks, and adds gate * y into an fp32 row accumulator; the last task to finish
-//            a 32-row chunk (atomic counter) rounds it to bf16, writes the output and re-zeroes the
-//            accumulator and counter for the next call (self-cleaning, no memset launch).
+//   routed unit (j, mt)   gate/up rows of slice mt (one 128-row m-tile: 64 gate + 64 up rows,
+//                         interleaved) of the j-th selected expert; CTA r of the pair holds the
+//                         input-column half r (H/128 blocks), and down-projection k-step mt for
+//                         output rows [H/2 * r, H/2 * (r + 1)) (H/256 blocks);
+//   shared unit (mt)      the same for the always-on shared expert.
 //
-// Each phase is a flat list of warp tasks (one weight-block slice each); task t runs on CTA
-// t % grid, so every SM carries a share and all of a phase's weight loads are in flight at once.
-// The down blocks of phase 2 are requested into L2 early (bulk L2 prefetch: the shared expert's
-// at kernel start, the routed experts' right after top-k), and each phase-2 warp issues its
-// weight loads before it builds act, so phase 2 mostly waits on L2, not HBM.  GEMV arithmetic as
-// in decode.cu.
-// Grid barrier: ever-growing arrival counters in the workspace; waits are bounded (1 s), on a
-// timeout the status word records it and moe_status resets the barrier state.
+// Per CTA the flow is:
+//   1. before the previous kernel in the stream has finished (programmatic dependent launch):
+//      bulk-copy the weights that do not depend on x -- the CTA's router rows (routed units) or
+//      its whole shared-expert share (shared units) -- into shared memory;
+//   2. stage x (fp32, and per 64-column group scaled by a power of two for the GEMVs);
+//   3. routed CTAs: compute their router logits and publish each as one 64-bit word
+//      (call tag << 32 | fp32 bits); every routed CTA polls all E words until they carry this
+//      call's tag -- data and synchronisation in one round trip, no grid barrier -- and picks the
+//      top k (every CTA gets the same answer); the CTA then bulk-copies its expert's gate/up half
+//      and down blocks (~110 KB) into shared memory in one wave;
+//   4. gate/up GEMV from shared memory as the copies land, the pair's two column halves summed
+//      through distributed shared memory, act = silu(G) * U for the 64 columns of the slice;
+//   5. down GEMV of the slice into the CTA's H/2 output rows, times the gate, added into an fp32
+//      row accumulator (vector reductions in L2); per 128-row chunk an arrival counter finds the
+//      last of the units, which rounds the chunk to bf16, writes it and re-zeroes the chunk's
+//      accumulator and counter (self-cleaning, no memset).
+// The shared-expert pairs never wait for routing.
+//
+// Call state lives in the workspace: a ticket counter every CTA increments at start (call number
+// = ticket / CTAs per call, so the router words of an earlier or abandoned call never carry the
+// current tag), the fp32 accumulator and the chunk counters (zero between calls), and a dirty
+// word that a CTA raises when one of its bounded waits runs out: the next call then zeroes the
+// accumulator and counters before anything is added, with no host intervention.
+//
+// GEMV arithmetic as in decode.cu: 4-bit codes enter the fp32 FMAs as subnormals (code * 2^-149),
+// the activations of each 64-column group are pre-scaled by a power of two, the scale is applied
+// once per (row, half group) and the bias as b * (sum of the half group's activations).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -31,38 +48,20 @@ namespace moe {
 
 namespace {
 
-constexpr int kFThreads = 512;
-constexpr int kFWarps = kFThreads / 32;
-constexpr int kGuKR = 4;   // k-ranges of the gate/up GEMV tasks
-constexpr int kDnKR = 4;   // k-ranges of the down GEMV tasks
+constexpr int kDThreads = 512;
+constexpr int kDWarps = kDThreads / 32;
+constexpr int kMaxRouterRows = 4;
+constexpr int kMaxDM = 12;           // down blocks per CTA (H / 256)
+constexpr int kMaxChunkBlocks = 8;   // gate/up blocks per landing chunk
 
 __device__ __forceinline__ float pow2f(int n) { return __int_as_float((127 + n) << 23); }
 __device__ __forceinline__ int group_exponent(float m) {
     int e = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
     return max(-126, min(100, e));
 }
+// position of element e8 (0..7 of an 8-column word) in the order the code bytes come out:
+// (word & 0x0F0F0F0F) yields columns {0,4,1,5}, ((word >> 4) & 0x0F0F0F0F) columns {2,6,3,7}
 __device__ __forceinline__ int slot_of(int e8) { return (e8 >> 2) | ((e8 & 3) << 1); }
-
-__device__ __forceinline__ float dot_group(const uint4& c0, const uint4& c1, const float* vp) {
-    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t m0 = w[i] & 0x0F0F0F0Fu;
-        const uint32_t m1 = (w[i] >> 4) & 0x0F0F0F0Fu;
-        const float4 x0 = *reinterpret_cast<const float4*>(vp + 8 * i);
-        const float4 x1 = *reinterpret_cast<const float4*>(vp + 8 * i + 4);
-        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4440)), x0.x, a0);
-        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4441)), x0.y, a1);
-        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4442)), x0.z, a0);
-        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m0, 0u, 0x4443)), x0.w, a1);
-        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4440)), x1.x, a0);
-        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4441)), x1.y, a1);
-        a0 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4442)), x1.z, a0);
-        a1 = fma_keep_subnormal(__uint_as_float(__byte_perm(m1, 0u, 0x4443)), x1.w, a1);
-    }
-    return a0 + a1;
-}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -74,378 +73,635 @@ __device__ __forceinline__ float warp_max(float v) {
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
-
-// Grid barrier on kBarCounters counters that only grow, 256 bytes apart: CTA b adds 1 (release,
-// GPU scope) to counter b mod kBarCounters, so few same-address atomics queue behind each other;
-// the barrier index follows from the value it found, and warp 0 then polls every counter (acquire)
-// until each has received one arrival per CTA mapped to it for this barrier.  No reset: between
-// barriers every counter holds a multiple of its CTA count (the handle zeroes them after a
-// timeout).  Bounded.
-constexpr int kBarCounters = 16;
-constexpr int kBarStride = 32;   // u64 words between counters
-
-__device__ bool grid_barrier(unsigned long long* ctr, unsigned nblocks, uint32_t* status, volatile int* abort_flag) {
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const unsigned nc = nblocks < (unsigned)kBarCounters ? nblocks : (unsigned)kBarCounters;
-        auto members = [&](unsigned j) { return nblocks / nc + (j < nblocks % nc ? 1u : 0u); };
-        unsigned long long b = 0;
-        if (lane == 0) {
-            const unsigned j = blockIdx.x % nc;
-            unsigned long long old;
-            asm volatile("atom.add.release.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr + (size_t)j * kBarStride) : "memory");
-            b = old / members(j);
-        }
-        b = __shfl_sync(0xffffffffu, b, 0);
-        bool ok = true;
-        if ((unsigned)lane < nc) {
-            const unsigned long long target = (b + 1) * members((unsigned)lane);
-            const unsigned long long* p = ctr + (size_t)lane * kBarStride;
-            const unsigned long long t0 = globaltimer_ns();
-            while (true) {
-                unsigned long long v;
-                asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-                if (v >= target) break;
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    set_status(status, MOE_STATUS_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        ok = __all_sync(0xffffffffu, ok);
-        if (lane == 0) *abort_flag = ok ? 0 : 1;
-    }
-    __syncthreads();
-    return *abort_flag == 0;
+// sum over the 16 lanes of each half warp (lanes 0-15 and 16-31 separately)
+__device__ __forceinline__ float half_warp_sum(float v) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
-// Order-preserving map of a float to an unsigned key (-0 first made +0, so equal floats give
-// equal keys).
 __device__ __forceinline__ uint32_t ord_key(float v) {
     const uint32_t u = __float_as_uint(v + 0.0f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-struct GemvTask {  // one warp: 32 rows (lane = row) of one m-tile, k-steps [k0, k1)
-    const uint8_t* blocks;  // first block of the m-tile
-    int row;                // block row of this lane
-    int k0, k1;
+// {a.x * b.x + c.x, a.y * b.y + c.y} in one packed fp32 FMA (sm_100), rounded once each, subnormal
+// operands kept (no .ftz): two of the GEMV's weight x activation products per instruction
+__device__ __forceinline__ float2 ffma2_keep_subnormal(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+        : "=l"(d)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+
+__device__ __forceinline__ float code_f(uint32_t m, uint32_t sel) { return __uint_as_float(__byte_perm(m, 0u, sel)); }
+
+// sum over the 32 columns of one half group: codes c (4 words), activations v in slot order
+__device__ __forceinline__ float dot32(const uint4& c, const float* v) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t m0 = w[i] & 0x0F0F0F0Fu;
+        const uint32_t m1 = (w[i] >> 4) & 0x0F0F0F0Fu;
+        const float4 x0 = *reinterpret_cast<const float4*>(v + 8 * i);
+        const float4 x1 = *reinterpret_cast<const float4*>(v + 8 * i + 4);
+        a = ffma2_keep_subnormal(make_float2(code_f(m0, 0x4440), code_f(m0, 0x4441)), make_float2(x0.x, x0.y), a);
+        b = ffma2_keep_subnormal(make_float2(code_f(m0, 0x4442), code_f(m0, 0x4443)), make_float2(x0.z, x0.w), b);
+        a = ffma2_keep_subnormal(make_float2(code_f(m1, 0x4440), code_f(m1, 0x4441)), make_float2(x1.x, x1.y), a);
+        b = ffma2_keep_subnormal(make_float2(code_f(m1, 0x4442), code_f(m1, 0x4443)), make_float2(x1.z, x1.w), b);
+    }
+    return (a.x + a.y) + (b.x + b.y);
+}
+
+// One comparator of the descending sort of a lane's (key, expert) pairs: the larger key first,
+// equal keys with the lower expert index first.
+__device__ __forceinline__ void cas_desc(uint32_t& ka, uint32_t& ia, uint32_t& kb, uint32_t& ib) {
+    const bool sw = kb > ka || (kb == ka && ib < ia);
+    const uint32_t k0 = sw ? kb : ka, i0 = sw ? ib : ia, k1 = sw ? ka : kb, i1 = sw ? ia : ib;
+    ka = k0; ia = i0; kb = k1; ib = i1;
+}
+
+// ---- cluster, memory-model and wait helpers ----------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// 16 bytes into the shared memory of the cluster CTA `rank`, at the offset of `local`, completing
+// 16 bytes of transaction count on that CTA's mbarrier at the offset of `local_bar`
+__device__ __forceinline__ void st_async_peer_v4(const float* local, const uint64_t* local_bar, uint32_t rank,
+                                                 float4 v) {
+    uint32_t ra, rb;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_u32(local_bar)), "r"(rank));
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(ra),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rb)
+                 : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Bounded wait for phase `parity` of an mbarrier (false after kWaitLimitNs).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// Shared-memory carve-up (byte offsets, computed on the host from DecodeGeom and checked there).
+struct Smem {
+    uint8_t* wgu;      // [KH][4608]  gate/up blocks: this unit's m-tile, input-column half r
+    uint8_t* wdn;      // [DM][4608]  down blocks: k-step mt of the CTA's DM output m-tiles
+    float* rrow;       // [R][H]      router rows of this CTA (routed units)
+    float* sgw;        // [H]         shared-expert gate vector (shared units and CTA 0)
+    float* xraw;       // [H]         x in fp32
+    float* xs;         // [H]         x pre-scaled per 64-column group, slot order
+    float* xsum;       // [H/32]      sum of x over each half group
+    float* xsc;        // [H/64]      2^(149-K) per group
+    float* part;       // [4][128]    gate/up partial row sums (block parity x column half)
+    float* mine;       // [128]       this CTA's gate/up row sums over its input-column half
+    float* peer;       // [128]       the partner's, written by the partner
+    float* act;        // [64]        act of the slice, pre-scaled, slot order
+    float* misc;       // [8]         asum[2], asc, gate, shared-gate dot, logits reduction ...
+    float* ydn;        // [2][DM*128] down partial sums by column half
+    float* logit;      // [256]
+    float* red;        // [kDWarps][kMaxRouterRows + 1] per-warp partial dots
+    int* ints;         // [16]        flags: abort, dirty, sel expert, chunk flags follow
+    uint64_t* bars;    // bar_r, bar_d, bar_x, bar_g[0..3]
 };
 
-// A task's codes and scale/bias words, loaded ahead of the arithmetic (up to 8 k-steps).
-struct GemvRegs {
-    uint4 a[8], b[8];
-    uint32_t sb[8];
-};
+__device__ __forceinline__ Smem carve(uint8_t* base, const DecodeGeom& g) {
+    Smem s;
+    s.wgu = base + g.off_wgu;
+    s.wdn = base + g.off_wdn;
+    s.rrow = reinterpret_cast<float*>(base + g.off_rrow);
+    s.sgw = reinterpret_cast<float*>(base + g.off_sgw);
+    s.xraw = reinterpret_cast<float*>(base + g.off_xraw);
+    s.xs = reinterpret_cast<float*>(base + g.off_xs);
+    s.xsum = reinterpret_cast<float*>(base + g.off_xsum);
+    s.xsc = reinterpret_cast<float*>(base + g.off_xsc);
+    s.part = reinterpret_cast<float*>(base + g.off_part);
+    s.mine = s.part + 4 * 128;
+    s.peer = s.mine + 128;
+    s.act = s.peer + 128;
+    s.misc = s.act + 64;
+    s.ydn = reinterpret_cast<float*>(base + g.off_ydn);
+    s.logit = reinterpret_cast<float*>(base + g.off_logit);
+    s.red = s.logit + 256;
+    s.ints = reinterpret_cast<int*>(s.red + kDWarps * (kMaxRouterRows + 1));
+    s.bars = reinterpret_cast<uint64_t*>(base + g.off_bars);
+    return s;
+}
 
-__device__ __forceinline__ void gemv_load(const GemvTask& t, GemvRegs& r) {
-    const int n = t.k1 - t.k0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        if (i < n) {
-            const uint8_t* blk = t.blocks + (size_t)(t.k0 + i) * kBlockBytes;
-            r.a[i] = __ldg(reinterpret_cast<const uint4*>(blk + t.row * 16));
-            r.b[i] = __ldg(reinterpret_cast<const uint4*>(blk + 2048 + t.row * 16));
-            r.sb[i] = __ldg(reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + t.row * 4));
+enum { kIntAbort = 0, kIntDirty = 1, kIntSel = 2, kIntTag = 3, kIntFlags = 4 };   // ints[4 + b]: chunk b finalised here
+enum { kMiscAsum0 = 0, kMiscAsum1 = 1, kMiscAsc = 2, kMiscGate = 3, kMiscSgDot = 4 };
+
+__global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, DecodeGeom g) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const Smem s = carve(smem_raw, g);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = c.H, E = c.E, k = c.k;
+    const int KSg = H / 64, MTd = H / 128, KSd = c.I / 64;
+    const uint32_t r = cluster_ctarank();
+    const int q = blockIdx.x >> 1;                      // work unit = cluster
+    const bool routed = q < k * g.MTg;
+    const int j = routed ? q / g.MTg : k;               // expert slot (k = the shared expert)
+    const int mt = routed ? q % g.MTg : q - k * g.MTg;  // 64-column slice of I
+    const int cr = blockIdx.x;                          // routed CTA index (routed units come first)
+    uint64_t* bar_r = s.bars;       // router rows and the shared-gate vector landed
+    uint64_t* bar_d = s.bars + 1;   // down blocks landed
+    uint64_t* bar_x = s.bars + 2;   // the partner's gate/up sums landed (st.async from the partner)
+    uint64_t* bar_g = s.bars + 3;   // gate/up chunks landed
+    const bool need_sg = c.has_shared && (!routed || blockIdx.x == 0);
+    int nrows = 0;   // router rows of this CTA
+    if (routed)
+        for (int i = 0; i < g.R; ++i) nrows += (cr + g.NR * i < E) ? 1 : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < 3 + g.nch; ++i) mbar_init(&s.bars[i], 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar_x, 128 * sizeof(float));   // before the partner can send (cluster barrier 1)
+        s.ints[kIntAbort] = 0;
+    }
+    cluster_arrive_relaxed();   // (1) this CTA has started; waited on before the first remote store
+    __syncthreads();
+
+    // ---- 1. weights that do not depend on x (nothing written by an earlier kernel is read yet)
+    // this unit's copies for expert e: the gate/up half in nch chunks (one thread), and the DM
+    // down blocks (one per lane of a warp, after lane 0 has set the barrier's byte count)
+    auto issue_gateup = [&](int e) {
+        const uint8_t* gu = c.w_gu + ((size_t)(e * g.MTg + mt) * KSg + (size_t)g.KH * r) * kBlockBytes;
+        for (int ch = 0; ch < g.nch; ++ch) {
+            const int b0 = ch * g.KH / g.nch, b1 = (ch + 1) * g.KH / g.nch;
+            mbar_arrive_expect_tx(&bar_g[ch], (uint32_t)((b1 - b0) * kBlockBytes));
+            bulk_g2s(s.wgu + (size_t)b0 * kBlockBytes, gu + (size_t)b0 * kBlockBytes, (uint32_t)((b1 - b0) * kBlockBytes),
+                     &bar_g[ch]);
         }
-    }
-}
-
-__device__ __forceinline__ float gemv_dot(const GemvTask& t, const GemvRegs& r, const float* vperm,
-                                          const float* vsum, const float* vsc) {
-    const int n = t.k1 - t.k0;
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        if (i < n) {
-            const int cc = t.k0 + i;
-            const float s = __half2float(__ushort_as_half((unsigned short)(r.sb[i] & 0xFFFFu)));
-            const float bb = __half2float(__ushort_as_half((unsigned short)(r.sb[i] >> 16)));
-            const float P = dot_group(r.a[i], r.b[i], vperm + 64 * cc);
-            acc += s * (P * vsc[cc]) + bb * vsum[cc];
+    };
+    auto issue_down = [&](int e) {   // called by a whole warp
+        if (lane == 0) mbar_arrive_expect_tx(bar_d, (uint32_t)(g.DM * kBlockBytes));
+        __syncwarp();
+        for (int b = lane; b < g.DM; b += 32) {
+            const int mtd = g.DM * (int)r + b;
+            bulk_g2s(s.wdn + (size_t)b * kBlockBytes, c.w_dn + ((size_t)(e * MTd + mtd) * KSd + mt) * kBlockBytes,
+                     kBlockBytes, bar_d);
         }
+    };
+    const bool need_r = nrows > 0 || need_sg;
+    if (need_r && warp == 2 && lane == 0) {
+        mbar_arrive_expect_tx(bar_r, (uint32_t)((nrows + (need_sg ? 1 : 0)) * H * sizeof(float)));
+        for (int i = 0; i < nrows; ++i)
+            bulk_g2s(s.rrow + (size_t)i * H, c.router32 + (size_t)(cr + g.NR * i) * H, (uint32_t)(H * sizeof(float)),
+                     bar_r);
+        if (need_sg) bulk_g2s(s.sgw, c.sgw, (uint32_t)(H * sizeof(float)), bar_r);
     }
-    return acc;
-}
-
-__device__ __forceinline__ float run_gemv(const GemvTask& t, const float* vperm, const float* vsum, const float* vsc) {
-    GemvRegs r;
-    gemv_load(t, r);   // every load of the task in flight before the arithmetic
-    return gemv_dot(t, r, vperm, vsum, vsc);
-}
-
-// One thread asks L2 to fetch the down blocks of (expert list entry, m-tile) chunks
-// blockIdx.x, blockIdx.x + gridDim.x, ...: one m-tile's whole k range is one contiguous run.
-// experts == nullptr stands for the shared expert (group E).  Not thread 0: its grid-barrier
-// release would wait for the prefetches to finish.
-__device__ __forceinline__ void prefetch_down(const Ctx& c, const int* experts, int nexp) {
-    if (threadIdx.x != 32) return;
-    const int MTd = c.H / 128, KSd = c.I / 64;
-    for (int ch = blockIdx.x; ch < nexp * MTd; ch += gridDim.x) {
-        const int e = experts ? experts[ch / MTd] : c.E, mt = ch % MTd;
-        prefetch_l2(c.w_dn + ((size_t)e * MTd + mt) * KSd * kBlockBytes, (uint32_t)(KSd * kBlockBytes));
+    if (!routed) {   // the shared expert is group E
+        if (warp == 0 && lane == 0) issue_gateup(E);
+        if (warp == 1) issue_down(E);
     }
-}
+    const float my_bias = (tid < nrows) ? c.rbias[cr + g.NR * tid] : 0.f;
+    bool wave_b = !routed;   // this CTA's unit copies are in flight (drained before exit)
 
-// Per-64-element group power-of-two scaling (see decode.cu): vperm in slot order, group sums, 2^(149-K).
-// One warp per group, 2 elements per lane; `src(i)` yields element i.
-template <typename F>
-__device__ __forceinline__ void stage_groups(int n, F src, float* vperm, float* vsum, float* vsc) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int grp = warp; grp < n / 64; grp += kFWarps) {
-        const float a0 = src(64 * grp + 2 * lane), a1 = src(64 * grp + 2 * lane + 1);
-        const float m = warp_max(fmaxf(fabsf(a0), fabsf(a1)));
-        const float s = warp_sum(a0 + a1);
+    // ---- 2. from here on x and the workspace are read: wait for the previous grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // x: 16-byte loads by the first H/8 threads; the call ticket and the dirty word are fetched
+    // by the last two warps at the same time (the tag is only needed at the router publish)
+    for (int i = tid; i < H / 8; i += kDThreads) {
+        const uint4 raw = reinterpret_cast<const uint4*>(c.x)[i];
+        reinterpret_cast<float4*>(s.xraw)[2 * i] =
+            make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u), __uint_as_float(raw.y << 16),
+                        __uint_as_float(raw.y & 0xFFFF0000u));
+        reinterpret_cast<float4*>(s.xraw)[2 * i + 1] =
+            make_float4(__uint_as_float(raw.z << 16), __uint_as_float(raw.z & 0xFFFF0000u), __uint_as_float(raw.w << 16),
+                        __uint_as_float(raw.w & 0xFFFF0000u));
+    }
+    if (tid == kDThreads - 64) {   // call tag: CTAs started before this one, over CTAs per call (+1)
+        const unsigned long long ticket = atomicAdd(c.dfz.ticket, 1ull);
+        s.ints[kIntTag] = (int)(uint32_t)(ticket / (unsigned long long)gridDim.x + 1ull);
+    }
+    if (tid == kDThreads - 32) s.ints[kIntDirty] = (int)ld_acquire_u32(c.dfz.dirty);
+    __syncthreads();
+    const uint32_t tag = (uint32_t)s.ints[kIntTag];
+    const bool dirty = s.ints[kIntDirty] != 0;
+    // per-group scaling of the input-column half this CTA's gate/up blocks cover
+    for (int grp = g.KH * (int)r + warp; grp < g.KH * ((int)r + 1); grp += kDWarps) {
+        const float a0 = s.xraw[64 * grp + 2 * lane], a1 = s.xraw[64 * grp + 2 * lane + 1];
+        const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(a0), fabsf(a1)))));
+        const float hs = half_warp_sum(a0 + a1);
         const int K = 125 - group_exponent(m);
         const float f1 = pow2f(K / 2), f2 = pow2f(K - K / 2);
         const int e0 = 2 * lane, e1 = 2 * lane + 1;
-        vperm[64 * grp + (e0 & ~7) + slot_of(e0 & 7)] = a0 * f1 * f2;
-        vperm[64 * grp + (e1 & ~7) + slot_of(e1 & 7)] = a1 * f1 * f2;
-        if (lane == 0) {
-            vsum[grp] = s;
-            vsc[grp] = pow2f(149 - K);
-        }
+        s.xs[64 * grp + (e0 & ~7) + slot_of(e0 & 7)] = a0 * f1 * f2;
+        s.xs[64 * grp + (e1 & ~7) + slot_of(e1 & 7)] = a1 * f1 * f2;
+        if ((lane & 15) == 0) s.xsum[2 * grp + (lane >> 4)] = hs;
+        if (lane == 0) s.xsc[grp] = pow2f(149 - K);
     }
-}
+    // a call after one that gave up part-way: the routed CTAs put the accumulator and the chunk
+    // counters back to zero (ordered before their router words by a fence)
+    if (dirty && routed) {
+        for (int i = cr * kDThreads + tid; i < H; i += g.NR * kDThreads) c.dfz.outacc[i] = 0.f;
+        for (int i = cr * kDThreads + tid; i < MTd; i += g.NR * kDThreads) c.dfz.cnt[i] = 0u;
+    }
 
-__global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(Ctx c) {
-    extern __shared__ __align__(16) float sm[];
-    const int H = c.H, I = c.I, E = c.E, k = c.k;
-    const int KSg = H / 64, MTg = I / 64;   // gate/up: k-steps, m-tiles
-    const int KSd = I / 64, MTd = H / 128;  // down
-    const int nslot = k + c.has_shared;
-    float* x32 = sm;                 // [H]
-    float* xperm = x32 + H;          // [H]
-    float* xsum = xperm + H;         // [H/64]
-    float* xsc = xsum + KSg;         // [H/64]
-    float* aperm = xsc + KSg;        // [I]
-    float* asum = aperm + I;         // [I/64]
-    float* asc = asum + KSd;         // [I/64]
-    float* logits = asc + KSd;       // [256]
-    float* red = logits + 256;       // [32]
-    int* sel = reinterpret_cast<int*>(red + 32);   // [32]
-    float* selg = reinterpret_cast<float*>(sel + 32);  // [33]: gates, then the shared gate
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(selg + 33);
-
-    float* rpart = c.dfz.rpart;      // [4][E]
-    float* gu = c.dfz.gu;            // [slots][kGuKR][2I]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = warp * gridDim.x + blockIdx.x;   // task t -> SM t % grid: a phase spreads over every SM
-    const int NW = gridDim.x * kFWarps;
-    const uint16_t* xr = c.x;        // T == 1
-
-    // ------------------------------------------------------------------ phase 0
-    if (c.has_shared) prefetch_down(c, nullptr, 1);   // the shared expert's down blocks, needed in phase 2
-    const int n_router = E * 4;
-    const int n_shared = c.has_shared ? MTg * 4 * kGuKR : 0;
-    const int hq = H / 4;   // router quarter row
-    // A warp's first task reads weights that do not depend on x: they are requested into L2 before
-    // x is staged, so the two memory latencies overlap (bulk L2 prefetch, lane 0 of the warp).
-    if (lane == 0) {
-        if (gw < n_router) {
-            prefetch_l2(c.router32 + (size_t)(gw >> 2) * H + (gw & 3) * hq, (uint32_t)(hq * sizeof(float)));
-        } else if (gw < n_router + n_shared) {
-            const int s0 = gw - n_router;
-            const int mt = s0 / (4 * kGuKR), q = (s0 / kGuKR) & 3, kr = s0 % kGuKR;
-            const int k0 = kr * KSg / kGuKR, k1 = (kr + 1) * KSg / kGuKR;
-            if (q == 0 && k1 > k0)   // the four row quarters share these blocks
-                prefetch_l2(c.w_gu + (((size_t)E * MTg + mt) * KSg + k0) * kBlockBytes, (uint32_t)((k1 - k0) * kBlockBytes));
-        }
-    }
-    // Launched as a programmatic dependent of the previous kernel in the stream: everything above
-    // reads only the handle's weights; x and the workspace are touched only after the previous
-    // grid has completed and its memory is visible.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (int i = threadIdx.x; i < H; i += kFThreads) x32[i] = __uint_as_float((uint32_t)xr[i] << 16);
-    if (threadIdx.x == 0) *abort_flag = 0;
-    __syncthreads();
-    stage_groups(H, [&](int i) { return x32[i]; }, xperm, xsum, xsc);
-    float sgd = 0.f;
-    if (c.has_shared)
-        for (int i = threadIdx.x; i < H; i += kFThreads) sgd = fmaf(x32[i], c.sgw[i], sgd);
-    sgd = warp_sum(sgd);
-    if (lane == 0) red[warp] = sgd;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float z = 0.f;
-        for (int w = 0; w < kFWarps; ++w) z += red[w];
-        selg[32] = c.has_shared ? 1.f / (1.f + expf(-z)) : 0.f;
-    }
-    for (int task = gw; task < n_router + n_shared; task += NW) {
-        if (task < n_router) {
-            const int e = task >> 2, kq = task & 3;
-            const float* wrow = c.router32 + (size_t)e * H + kq * hq;
-            float d = 0.f;
-#pragma unroll 4
-            for (int h = lane * 4; h < hq; h += 128) {
-                const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + h));
-                const float4 xv = *reinterpret_cast<const float4*>(x32 + kq * hq + h);
-                d = fmaf(wv.x, xv.x, fmaf(wv.y, xv.y, fmaf(wv.z, xv.z, fmaf(wv.w, xv.w, d))));
-            }
-            d = warp_sum(d);
-            if (lane == 0) rpart[kq * E + e] = d;
-        } else {
-            const int s = task - n_router;
-            const int mt = s / (4 * kGuKR), q = (s / kGuKR) & 3, kr = s % kGuKR;
-            GemvTask t;
-            t.blocks = c.w_gu + ((size_t)E * MTg + mt) * KSg * kBlockBytes;   // shared expert = group E
-            t.row = 32 * q + lane;
-            t.k0 = kr * KSg / kGuKR;
-            t.k1 = (kr + 1) * KSg / kGuKR;
-            const float v = run_gemv(t, xperm, xsum, xsc);
-            gu[((size_t)k * kGuKR + kr) * (2 * I) + mt * 128 + t.row] = v;
-        }
-    }
-    if (!grid_barrier(c.dfz.bar, gridDim.x, c.status, abort_flag)) return;
-
-    // ------------------------------------------------------------------ phase 1: top-k, routed gate/up
-    for (int e = threadIdx.x; e < 256; e += kFThreads) {
-        float v = -INFINITY;
-        if (e < E) {
-            const float s = rpart[e] + rpart[E + e] + rpart[2 * E + e] + rpart[3 * E + e] + c.rbias[e];
-            v = (s != s) ? -INFINITY : s;
-        }
-        logits[e] = v;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        // top-k by logit, ties to the lower expert index: per round one warp-wide max of the keys
-        // and one min of the indices holding it (two redux instructions)
-        uint32_t key[8];
+    // ---- 3. router logits and the shared gate sigmoid(x . w_sg) (the shared units' combine
+    // weight; CTA 0 also reports it)
+    bool ok = true;
+    if (need_r) ok = wait_bar(bar_r, 0);
+    {
+        float acc[kMaxRouterRows];
+        float d = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) key[i] = ord_key(logits[lane + 32 * i]);
-        unsigned taken = 0;
-        int my_e = 0;
-        float my_v = 0.f;
-        for (int j = 0; j < k; ++j) {
-            uint32_t best = 0;
-            int bi = -1;
+        for (int i = 0; i < kMaxRouterRows; ++i) acc[i] = 0.f;
+        if (ok) {
+            for (int h = tid; h < H; h += kDThreads) {
+                const float xv = s.xraw[h];
+#pragma unroll
+                for (int i = 0; i < kMaxRouterRows; ++i)
+                    if (i < nrows) acc[i] = fmaf(xv, s.rrow[(size_t)i * H + h], acc[i]);
+                if (need_sg) d = fmaf(xv, s.sgw[h], d);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kMaxRouterRows; ++i) {
+            if (i < nrows) {   // uniform across the CTA
+                const float v = warp_sum(acc[i]);
+                if (lane == 0) s.red[kDWarps + warp * kMaxRouterRows + i] = v;
+            }
+        }
+        if (need_sg) {
+            d = warp_sum(d);
+            if (lane == 0) s.red[warp] = d;
+        }
+    }
+    if (__syncthreads_or(!ok)) {
+        ok = false;
+        if (tid == 0) {
+            set_status(c.status, MOE_STATUS_TIMEOUT);
+            atomicOr(c.dfz.dirty, 1u);
+        }
+    }
+    if (routed && ok && tid < nrows) {
+        const int e = cr + g.NR * tid;
+        float z = 0.f;
+        for (int w = 0; w < kDWarps; ++w) z += s.red[kDWarps + w * kMaxRouterRows + tid];
+        z += my_bias;
+        const bool stall = (c.flags & 0x100u) && cr == 0 && tag == 1u;   // test only: first call withholds
+        // the word carries its own data; after a failed call it must also follow this CTA's zeroing
+        if (dirty) fence_acq_rel_gpu();
+        if (!stall) st_relaxed_u64(c.dfz.slots + e, ((unsigned long long)tag << 32) | __float_as_uint(z));
+    }
+    if (need_sg && tid == 32) {
+        float zz = 0.f;
+        for (int w = 0; w < kDWarps; ++w) zz += s.red[w];
+        s.misc[kMiscSgDot] = 1.f / (1.f + expf(-zz));
+    }
+    if (ok && (routed || dirty) && warp == 0) {
+        // every router word of this call: relaxed polls (each word carries its data; no load is
+        // left in flight when the loop ends)
+        uint32_t key[8], idx[8];
+        float lg[8];
+        const unsigned long long t0 = globaltimer_ns();
+        while (true) {
+            unsigned long long cur[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cur[i] = (lane + 32 * i < E) ? ld_relaxed_u64(c.dfz.slots + lane + 32 * i) : 0ull;
+            bool all = true;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                if (lane + 32 * i < E && !((taken >> i) & 1u) && (bi < 0 || key[i] > best)) { best = key[i]; bi = i; }
+                const int e = lane + 32 * i;
+                const float f = __uint_as_float((uint32_t)cur[i]);
+                lg[i] = (e < E && f == f) ? f : -INFINITY;
+                if (e < E && (uint32_t)(cur[i] >> 32) != tag) all = false;
             }
-            const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-            const uint32_t cand = (bi >= 0 && best == m) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
-            const uint32_t be = __reduce_min_sync(0xffffffffu, cand);
-            if ((int)(be & 31u) == lane) taken |= 1u << (be >> 5);
-            if (lane == j) { my_e = (int)be; my_v = logits[be & 255u]; }
+            if (__all_sync(0xffffffffu, all)) break;
+            if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {   // one decision for the warp
+                ok = false;
+                break;
+            }
         }
-        const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-        const float p = lane < k ? expf(my_v - vmax) : 0.f;
-        const float z = warp_sum(p);
-        if (lane < k) {
-            if (my_e < 0 || my_e >= E) { set_status(c.status, MOE_STATUS_BOUNDS); my_e = 0; }
-            sel[lane] = my_e;
-            selg[lane] = p / z;
-            if (blockIdx.x == 0) {
+        ok = __all_sync(0xffffffffu, ok);
+        if (dirty) fence_acq_rel_gpu();   // every routed CTA's zeroing precedes what follows
+        if (ok && routed) {
+            // top k by logit, ties to the lower expert index: each lane sorts its 8 (key, expert)
+            // pairs once (19-comparator network), then every pick is the lanes' heads' maximum
+            // key, the lowest expert among the heads holding it, and a pop of the winner's head
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane + 32 * i;
+                key[i] = e < E ? ord_key(lg[i]) : 0u;
+                idx[i] = e < E ? (uint32_t)e : 0xFFFFFFFFu;
+            }
+            cas_desc(key[0], idx[0], key[2], idx[2]); cas_desc(key[1], idx[1], key[3], idx[3]);
+            cas_desc(key[4], idx[4], key[6], idx[6]); cas_desc(key[5], idx[5], key[7], idx[7]);
+            cas_desc(key[0], idx[0], key[4], idx[4]); cas_desc(key[1], idx[1], key[5], idx[5]);
+            cas_desc(key[2], idx[2], key[6], idx[6]); cas_desc(key[3], idx[3], key[7], idx[7]);
+            cas_desc(key[0], idx[0], key[1], idx[1]); cas_desc(key[2], idx[2], key[3], idx[3]);
+            cas_desc(key[4], idx[4], key[5], idx[5]); cas_desc(key[6], idx[6], key[7], idx[7]);
+            cas_desc(key[2], idx[2], key[4], idx[4]); cas_desc(key[3], idx[3], key[5], idx[5]);
+            cas_desc(key[1], idx[1], key[4], idx[4]); cas_desc(key[3], idx[3], key[6], idx[6]);
+            cas_desc(key[1], idx[1], key[2], idx[2]); cas_desc(key[3], idx[3], key[4], idx[4]);
+            cas_desc(key[5], idx[5], key[6], idx[6]);
+            int my_e = 0;
+            for (int jj = 0; jj < k; ++jj) {
+                const uint32_t mx = __reduce_max_sync(0xffffffffu, key[0]);
+                const uint32_t be = __reduce_min_sync(0xffffffffu, key[0] == mx ? idx[0] : 0xFFFFFFFFu);
+                if (idx[0] == be) {   // pop the winner's head
+#pragma unroll
+                    for (int i = 0; i < 7; ++i) { key[i] = key[i + 1]; idx[i] = idx[i + 1]; }
+                    key[7] = 0u;
+                    idx[7] = 0xFFFFFFFFu;
+                }
+                if (lane == jj) my_e = (int)be;
+            }
+            // lane jj < k fetches the logit of its pick from the lane that holds it
+            float my_v = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float cv = __shfl_sync(0xffffffffu, lg[i], my_e & 31);
+                if ((my_e >> 5) == i) my_v = cv;
+            }
+            const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+            const float p = lane < k ? expf(my_v - vmax) : 0.f;
+            const float zsum = warp_sum(p);
+            if (lane < k && (my_e < 0 || my_e >= E)) {
+                set_status(c.status, MOE_STATUS_BOUNDS);
+                my_e = 0;
+            }
+            const int sel = __shfl_sync(0xffffffffu, my_e, j);
+            const float gsel = __shfl_sync(0xffffffffu, p, j) / zsum;
+            if (lane == 0) {
+                s.ints[kIntSel] = sel;
+                s.misc[kMiscGate] = gsel;
+                issue_gateup(sel);   // at once: the rest of the CTA learns the expert after a barrier
+            }
+            if (blockIdx.x == 0 && lane < k) {
                 c.idx[lane] = my_e;
-                c.gates[lane] = p / z;
+                c.gates[lane] = p / zsum;
             }
         }
-        if (blockIdx.x == 0 && lane == 0) c.sg[0] = selg[32];
+        if (lane == 0 && !ok) {
+            set_status(c.status, MOE_STATUS_TIMEOUT);
+            atomicOr(c.dfz.dirty, 1u);
+        }
+        if (lane == 0) s.ints[kIntAbort] = ok ? 0 : 1;
     }
     __syncthreads();
-    prefetch_down(c, sel, k);   // the routed experts' down blocks stream into L2 during gate/up
-    {
-        const int n_tasks = k * MTg * 4 * kGuKR;
-        for (int task = gw; task < n_tasks; task += NW) {
-            const int j = task / (MTg * 4 * kGuKR);
-            const int r = task % (MTg * 4 * kGuKR);
-            const int mt = r / (4 * kGuKR), q = (r / kGuKR) & 3, kr = r % kGuKR;
-            GemvTask t;
-            t.blocks = c.w_gu + ((size_t)sel[j] * MTg + mt) * KSg * kBlockBytes;
-            t.row = 32 * q + lane;
-            t.k0 = kr * KSg / kGuKR;
-            t.k1 = (kr + 1) * KSg / kGuKR;
-            const float v = run_gemv(t, xperm, xsum, xsc);
-            gu[((size_t)j * kGuKR + kr) * (2 * I) + mt * 128 + t.row] = v;
-        }
+    ok = ok && s.ints[kIntAbort] == 0;
+    if (routed && ok && warp == 1) issue_down(s.ints[kIntSel]);
+    if (routed && ok) wave_b = true;
+    if (!routed && tid == 0) s.misc[kMiscGate] = s.misc[kMiscSgDot];
+    if (blockIdx.x == 0 && tid == 32) {
+        c.sg[0] = c.has_shared ? s.misc[kMiscSgDot] : 0.f;
+        if (ok && dirty) st_release_u32(c.dfz.dirty, 0u);   // every routed CTA has read it
     }
-    if (!grid_barrier(c.dfz.bar, gridDim.x, c.status, abort_flag)) return;
-    // the next kernel in the stream may be scheduled from here on (its CTAs take an SM as this
-    // grid's CTAs leave it, and wait for this grid's completion before reading anything it writes)
+    // the next kernel in the stream may be scheduled from here on (it waits for this grid's
+    // completion before it reads anything this grid writes)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    // ------------------------------------------------------------------ phase 2: down + combine
-    const int tasks_per_slot = MTd * 4 * kDnKR;
-    const int blocks_per_slot = (tasks_per_slot + kFWarps - 1) / kFWarps;
-    const int expected = nslot * kDnKR;
-    for (int vb = blockIdx.x; vb < nslot * blocks_per_slot; vb += gridDim.x) {
-        const int j = vb % nslot, bi = vb / nslot;
-        const int e = (j < k) ? sel[j] : E;
-        const float gate = (j < k) ? selg[j] : selg[32];
-        const int task = bi * kFWarps + warp;
-        GemvTask t;
-        GemvRegs wr;
-        if (task < tasks_per_slot) {   // weight loads first: they overlap the act staging below
-            const int mt = task / (4 * kDnKR), q = (task / kDnKR) & 3, kr = task % kDnKR;
-            t.blocks = c.w_dn + ((size_t)e * MTd + mt) * KSd * kBlockBytes;
-            t.row = 32 * q + lane;
-            t.k0 = kr * KSd / kDnKR;
-            t.k1 = (kr + 1) * KSd / kDnKR;
-            gemv_load(t, wr);
-        }
-        __syncthreads();
-        // act = silu(G) * U for this slot, from the k-range partials (gate row / up row of column i)
-        stage_groups(I, [&](int i) {
-            const int mt = i >> 6, il = i & 63, q = il >> 4, li = il & 15;
-            const int rg = mt * 128 + 32 * q + li, ru = rg + 16;
-            float G = 0.f, U = 0.f;
+    // ---- 4. gate/up GEMV over this CTA's input-column half, as the chunks land
+    const int row = tid & 127, hh = (tid >> 7) & 1, par = tid >> 8;
+    float acc = 0.f;
+    bool wok = ok;
+    if (ok) {
+        for (int ch = 0; ch < g.nch; ++ch) {
+            if (!wait_bar(&bar_g[ch], 0)) { wok = false; break; }
+            const int b0 = ch * g.KH / g.nch, b1 = (ch + 1) * g.KH / g.nch;
 #pragma unroll
-            for (int kr = 0; kr < kGuKR; ++kr) {
-                G += gu[((size_t)j * kGuKR + kr) * (2 * I) + rg];
-                U += gu[((size_t)j * kGuKR + kr) * (2 * I) + ru];
-            }
-            return G * U / (1.f + expf(-G));
-        }, aperm, asum, asc);
-        __syncthreads();
-        if (task < tasks_per_slot) {
-            const int mt = task / (4 * kDnKR), q = (task / kDnKR) & 3;
-            const float y = gemv_dot(t, wr, aperm, asum, asc) * gate;
-            const int h = mt * 128 + t.row;
-            atomicAdd(&c.dfz.outacc[h], y);
-            __syncwarp();
-            unsigned last = 0;
-            if (lane == 0) {
-                // acq_rel: releases this warp's additions, and the last arriver acquires everyone's
-                unsigned old;
-                asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(&c.dfz.cnt[mt * 4 + q]) : "memory");
-                last = old == (unsigned)expected - 1 ? 1u : 0u;
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            __syncwarp();
-            if (last) {
-                const float v = atomicExch(&c.dfz.outacc[h], 0.f);
-                c.out[h] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                if (lane == 0) atomicExch(&c.dfz.cnt[mt * 4 + q], 0u);
+            for (int i = 0; i < kMaxChunkBlocks / 2; ++i) {
+                const int b = b0 + par + 2 * i;
+                if (b < b1) {
+                    const int kc = g.KH * (int)r + b;   // 64-column group of x
+                    const uint8_t* blk = s.wgu + (size_t)b * kBlockBytes;
+                    const uint4 cw = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
+                    const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+                    const float P = dot32(cw, s.xs + 64 * kc + 32 * hh);
+                    const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+                    const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
+                    acc += sc * (P * s.xsc[kc]) + bi * s.xsum[2 * kc + hh];
+                }
             }
         }
     }
+    s.part[(par * 2 + hh) * 128 + row] = acc;
+    if (__syncthreads_or(!wok)) ok = false;
+    if (ok && tid < 128) s.mine[tid] = (s.part[tid] + s.part[128 + tid]) + (s.part[256 + tid] + s.part[384 + tid]);
+    cluster_wait();   // (1) the partner has started (its exchange mbarrier expects our 512 bytes)
+    __syncthreads();
+    // the pair's exchange: this CTA's 128 row sums go into the partner's shared memory with
+    // asynchronous remote stores that complete the partner's mbarrier; each CTA waits on its own.
+    // A CTA that gave up still waits for its partner's sums (bounded), so neither exits while the
+    // other may still be writing into it.
+    if (ok && tid < 32)
+        st_async_peer_v4(s.peer + 4 * tid, bar_x, r ^ 1u, reinterpret_cast<const float4*>(s.mine)[tid]);
+    if (!wait_bar(bar_x, 0)) ok = false;
+    if (__syncthreads_or(!ok)) ok = false;
+
+    // act = silu(G) * U for the slice's 64 columns: G and U of column i are rows 32(i/16) + i%16
+    // and 16 rows further of the interleaved m-tile; pre-scaled for the down GEMV
+    if (ok && warp == 0) {
+        float a[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = 2 * lane + u;
+            const int rg = 32 * (i >> 4) + (i & 15), ru = rg + 16;
+            const float G = s.mine[rg] + s.peer[rg], U = s.mine[ru] + s.peer[ru];
+            a[u] = G * U / (1.f + expf(-G));
+        }
+        const float m = warp_max(fmaxf(fabsf(a[0]), fabsf(a[1])));
+        const float hs = half_warp_sum(a[0] + a[1]);
+        const int K = 125 - group_exponent(m);
+        const float f1 = pow2f(K / 2), f2 = pow2f(K - K / 2);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = 2 * lane + u;
+            s.act[(i & ~7) + slot_of(i & 7)] = a[u] * f1 * f2;
+        }
+        if ((lane & 15) == 0) s.misc[kMiscAsum0 + (lane >> 4)] = hs;
+        if (lane == 0) s.misc[kMiscAsc] = pow2f(149 - K);
+    }
+    bool dok = ok;
+    if (ok) dok = wait_bar(bar_d, 0);
+    if (__syncthreads_or(!dok)) ok = false;
+
+    // ---- 5. down GEMV: DM output m-tiles x 128 rows x this slice's 64 columns
+    if (ok) {
+        float4 av[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) av[i] = reinterpret_cast<const float4*>(s.act + 32 * hh)[i];
+        const float asc = s.misc[kMiscAsc], asum = s.misc[kMiscAsum0 + hh];
+        // this thread's (up to kMaxDM / 2) blocks: every shared-memory load first, then the math
+        uint4 cw[kMaxDM / 2];
+        uint32_t sb[kMaxDM / 2];
+#pragma unroll
+        for (int i = 0; i < kMaxDM / 2; ++i) {
+            const int b = par + 2 * i;
+            if (b < g.DM) {
+                const uint8_t* blk = s.wdn + (size_t)b * kBlockBytes;
+                cw[i] = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
+                sb[i] = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kMaxDM / 2; ++i) {
+            const int b = par + 2 * i;
+            if (b < g.DM) {
+                const float P = dot32(cw[i], reinterpret_cast<const float*>(av));
+                const float sc = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
+                const float bi = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
+                s.ydn[hh * g.DM * 128 + b * 128 + row] = sc * (P * asc) + bi * asum;
+            }
+        }
+    }
+    __syncthreads();
+    if (ok) {
+        const float gate = s.misc[kMiscGate];
+        const int nrow = g.DM * 128;
+        float* dst = c.dfz.outacc + (size_t)g.DM * r * 128;
+        for (int i4 = tid; 4 * i4 < nrow; i4 += kDThreads) {
+            const float4 y0 = reinterpret_cast<const float4*>(s.ydn)[i4];
+            const float4 y1 = reinterpret_cast<const float4*>(s.ydn + nrow)[i4];
+            red_add_v4(dst + 4 * i4, (y0.x + y1.x) * gate, (y0.y + y1.y) * gate, (y0.z + y1.z) * gate,
+                       (y0.w + y1.w) * gate);
+        }
+    }
+    __syncthreads();
+    // one arrival per 128-row chunk; the last of the units finalises the chunk
+    if (ok && tid < g.DM) {
+        const int mtd = g.DM * (int)r + tid;
+        const unsigned old = atom_add_acq_rel(c.dfz.cnt + mtd, 1u);
+        s.ints[kIntFlags + tid] = (old == (unsigned)(g.units - 1)) ? 1 : 0;
+    }
+    __syncthreads();
+    if (ok) {
+        for (int i = tid; i < g.DM * 128; i += kDThreads) {
+            if (!s.ints[kIntFlags + (i >> 7)]) continue;
+            const size_t hrow = (size_t)g.DM * r * 128 + i;
+            const float v = atomicExch(c.dfz.outacc + hrow, 0.f);
+            c.out[hrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
+        if (tid < g.DM && s.ints[kIntFlags + tid]) atomicExch(c.dfz.cnt + g.DM * (int)r + tid, 0u);
+    }
+    if (!ok && tid == 0) {
+        set_status(c.status, MOE_STATUS_TIMEOUT);
+        atomicOr(c.dfz.dirty, 1u);
+    }
+    // nothing may still be landing in this CTA's shared memory when it exits
+    if (tid == 0) {
+        if (need_r) mbar_drain(bar_r, 0);
+        if (wave_b) {
+            for (int ch = 0; ch < g.nch; ++ch) mbar_drain(&bar_g[ch], 0);
+            mbar_drain(bar_d, 0);
+        }
+    }
+    __syncthreads();
 }
 
 }  // namespace
 
-int decode_fused_smem_bytes(int H, int I) {
-    return (int)sizeof(float) * (2 * H + 2 * (H / 64) + I + 2 * (I / 64) + 256 + 32 + 32 + 33 + 4);
+// Launch geometry of the fused kernel for a layer shape, or false when the shape does not fit it
+// (the multi-kernel GEMV chain then serves batch-1 decode).
+bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeom* out) {
+    DecodeGeom g{};
+    if (H % 256 != 0 || I % 64 != 0) return false;
+    g.MTg = I / 64;
+    g.units = (k + has_shared) * g.MTg;
+    g.NR = 2 * k * g.MTg;
+    g.R = (E + g.NR - 1) / g.NR;
+    if (g.R > kMaxRouterRows) return false;
+    g.KH = H / 128;
+    g.nch = g.KH < 4 ? g.KH : 4;
+    g.DM = H / 256;
+    if (g.DM > kMaxDM) return false;   // also bounds the chunk flags in the ints area
+    if ((g.KH + g.nch - 1) / g.nch > kMaxChunkBlocks) return false;
+    auto al = [](size_t v) { return (v + 127) / 128 * 128; };
+    size_t o = 0;
+    g.off_wgu = o; o = al(o + (size_t)g.KH * kBlockBytes);
+    g.off_wdn = o; o = al(o + (size_t)g.DM * kBlockBytes);
+    g.off_rrow = o; o = al(o + sizeof(float) * (size_t)g.R * H);
+    g.off_sgw = o; o = al(o + sizeof(float) * (size_t)H);
+    g.off_xraw = o; o = al(o + sizeof(float) * (size_t)H);
+    g.off_xs = o; o = al(o + sizeof(float) * (size_t)H);
+    g.off_xsum = o; o = al(o + sizeof(float) * (size_t)(H / 32));
+    g.off_xsc = o; o = al(o + sizeof(float) * (size_t)(H / 64));
+    g.off_part = o; o = al(o + sizeof(float) * (4 * 128 + 128 + 128 + 64 + 8));
+    g.off_ydn = o; o = al(o + sizeof(float) * 2 * (size_t)g.DM * 128);
+    g.off_logit = o; o = al(o + sizeof(float) * (256 + kDWarps * (kMaxRouterRows + 1)) + sizeof(int) * 16);
+    g.off_bars = o; o = al(o + sizeof(uint64_t) * 7);
+    g.smem = (int)o;
+    if (g.smem > 227 * 1024) return false;
+    *out = g;
+    return true;
 }
 
-cudaError_t launch_decode_fused(const Ctx& c, int num_sms, cudaStream_t st) {
-    const int smem = decode_fused_smem_bytes(c.H, c.I);
+cudaError_t decode_fused_prepare(const DecodeGeom& g) {
+    return cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem);
+}
+
+// Clusters of the fused kernel that fit on the device at once (all must be resident together).
+cudaError_t decode_fused_max_clusters(const DecodeGeom& g, int* n) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(num_sms);
-    cfg.blockDim = dim3(kFThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3(2 * g.units);
+    cfg.blockDim = dim3(kDThreads);
+    cfg.dynamicSmemBytes = g.smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(n, decode_fused_kernel, &cfg);
+}
+
+cudaError_t launch_decode_fused(const Ctx& c, const DecodeGeom& g, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * g.units);
+    cfg.blockDim = dim3(kDThreads);
+    cfg.dynamicSmemBytes = g.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlaps the launch with the previous kernel's tail
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, decode_fused_kernel, c);
+    return cudaLaunchKernelEx(&cfg, decode_fused_kernel, c, g);
 }
 
 }  // namespace moe

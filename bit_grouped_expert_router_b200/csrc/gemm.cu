@@ -108,6 +108,8 @@ __device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c, int bn) {
 template <bool GATEUP, int CTAS>
 __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
     grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps) {
+    griddep_wait();
+    griddep_launch_dependents();
     using K = GemmCfg<CTAS>;
     constexpr int kBN = K::kBN, kEpiWarps = K::kEpiWarps, kTransformWarps = K::kTransformWarps;
     constexpr int kEpiWarp0 = K::kEpiWarp0, kTmemCols = K::kTmemCols, kAccCols = K::kAccCols;
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 const bool from_x = GATEUP && c.has_shared && tile.x == c.E;   // shared expert: token order
                 const CUtensorMap* map = &maps.m[from_x ? 1 : 0][hsel];
                 const int y = from_x ? tile.y - shared_base : tile.y;
-                const uint32_t b_bytes = (uint32_t)(64 << hsel) * 128;
+                const uint32_t b_bytes = (uint32_t)token_box_rows(hsel) * 128;
                 const uint8_t* wsrc = wbase + ((size_t)tile.x * MT + mt) * KS * kBlockBytes;
                 for (int kc = 0; kc < KS; ++kc) {
                     int ok = 1;
@@ -426,6 +428,8 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
 
 // xp[p] = x16[row_token[p]] for the T*k routed bucket rows: one warp per row, 16-byte copies.
 __global__ void __launch_bounds__(256) gather_rows_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int lane = lane_id();
     const int nrows = c.T * c.k;
     for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < nrows; p += gridDim.x * 8) {
@@ -463,8 +467,7 @@ cudaError_t launch_grouped(const Ctx& c, const TokenMaps& maps, int num_sms, cud
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, CTAS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmemBytes);
     if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<GATEUP, CTAS><<<num_sms * CTAS, K::kThreads, K::kSmemBytes, st>>>(c, maps);
-    return cudaGetLastError();
+    return launch_pdl(grouped_gemm_kernel<GATEUP, CTAS>, dim3(num_sms * CTAS), dim3(K::kThreads), K::kSmemBytes, st, c, maps);
 }
 
 }  // namespace
@@ -474,8 +477,7 @@ int gemm_tile_rows(int T, int k, int E) { return T * k <= 64 * E ? GemmCfg<2>::k
 cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st) {
     const int rows = c.T * c.k;
     const int blocks = max(1, min((rows + 7) / 8, num_sms * 8));
-    gather_rows_kernel<<<blocks, 256, 0, st>>>(c);
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, c);
 }
 
 // The tile list (built for c.tile_rows rows per tile) selects the launch shape.
@@ -493,6 +495,8 @@ cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, c
 
 // out[t][h] = bf16(acc[t][h]), round to nearest even; 8 elements per thread per step.
 __global__ void __launch_bounds__(256) finalize_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     const size_t n8 = (size_t)c.T * c.H / 8;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
         const float4 a = reinterpret_cast<const float4*>(c.acc)[2 * i];
@@ -513,8 +517,7 @@ cudaError_t launch_finalize(const Ctx& c, cudaStream_t st) {
     // one 8-element chunk per thread (the loop only covers grids past the launch limit)
     const size_t want = (n8 + 255) / 256;
     const int blocks = (int)(want < (size_t)(1u << 30) ? want : (size_t)(1u << 30));
-    finalize_kernel<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(c);
-    return cudaGetLastError();
+    return launch_pdl(finalize_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st, c);
 }
 
 }  // namespace moe

@@ -31,15 +31,26 @@ struct RepackArgs {
     uint32_t* inexact;
 };
 
-// Workspace of the fused batch-1 decode kernel.  outacc and cnt are zero between calls (the
-// kernel re-zeroes what it used); bar holds grid-barrier arrival counts (between calls each a
-// multiple of the number of CTAs that arrive on it).
+// Workspace of the fused batch-1 decode kernel (zero when the handle is created).
 struct DecodeFusedWs {
-    float* rpart;    // [4][E] quarter-row router partial logits
-    float* gu;       // [k+1][4][2I] gate/up k-range partial sums
-    float* outacc;   // [H] fp32 output accumulator
-    unsigned* cnt;   // [H/32] arrivals per 32-row output chunk
-    unsigned long long* bar;   // [16 x 32] grid-barrier arrival counters (256 B apart), only ever incremented
+    unsigned long long* ticket;   // [1] CTAs started, over all calls (call number = ticket / CTAs per call)
+    unsigned long long* slots;    // [E] router logit of expert e as (call tag << 32) | fp32 bits
+    float* outacc;                // [H] fp32 output accumulator; zero between calls
+    unsigned* cnt;                // [H/128] unit arrivals per 128-row output chunk; zero between calls
+    unsigned* dirty;              // [1] raised by a call that gave up part-way; the next call resets
+};
+
+// Launch geometry and shared-memory carve-up of the fused batch-1 decode kernel (host-computed).
+struct DecodeGeom {
+    int MTg;      // 64-column slices of I (gate/up m-tiles of 128 interleaved rows)
+    int units;    // (k + has_shared) * MTg work units, one 2-CTA cluster each
+    int NR;       // routed CTAs (2 * k * MTg): router rows are dealt to them
+    int R;        // router rows per routed CTA (ceil(E / NR))
+    int KH;       // gate/up blocks per CTA (H / 128: one input-column half)
+    int nch;      // landing chunks of the gate/up copy
+    int DM;       // down blocks per CTA (H / 256 output m-tiles)
+    int smem;     // dynamic shared memory bytes
+    size_t off_wgu, off_wdn, off_rrow, off_sgw, off_xraw, off_xs, off_xsum, off_xsc, off_part, off_ydn, off_logit, off_bars;
 };
 
 // Everything a forward-path kernel needs (passed by value).
@@ -82,7 +93,6 @@ struct Ctx {
     float* dact;
     float* dscale;
     uint32_t* status;
-    unsigned int* counters;
     DecodeFusedWs dfz;
 };
 
@@ -101,7 +111,12 @@ cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
 cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st);
 
-// Token-tile TMA maps of one grouped GEMM: m[source][h] with box {64 columns, 64 << h rows}.
+// Rows of the token-tile TMA box with selector h: 64, 128 or 256 (a tile of n tokens loads the
+// smallest box that holds n rows; the one-CTA GEMM shape has tiles of up to 256 tokens, the
+// two-CTA shape 128).
+__host__ __device__ constexpr int token_box_rows(int h) { return 64 << h; }
+
+// Token-tile TMA maps of one grouped GEMM: m[source][h] with box {64 columns, token_box_rows(h) rows}.
 // gate/up: source 0 = bucketed rows xp, source 1 = the activations x16 (shared expert);
 // down: source 0 = act (source 1 unused).
 struct TokenMaps {
@@ -121,8 +136,10 @@ int gemm_tile_rows(int T, int k, int E);
 void set_last_error(const char* msg);
 
 // decode sparse GEMV
-cudaError_t launch_decode_fused(const Ctx& c, int num_sms, cudaStream_t st);
-int decode_fused_smem_bytes(int H, int I);
+bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeom* out);
+cudaError_t decode_fused_prepare(const DecodeGeom& g);
+cudaError_t decode_fused_max_clusters(const DecodeGeom& g, int* n);
+cudaError_t launch_decode_fused(const Ctx& c, const DecodeGeom& g, cudaStream_t st);
 cudaError_t launch_gemv_gateup(const Ctx& c, cudaStream_t st);
 cudaError_t launch_gemv_down(const Ctx& c, cudaStream_t st);
 

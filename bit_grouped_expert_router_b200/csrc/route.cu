@@ -26,6 +26,8 @@ namespace moe {
 // coalesced row read shared by TT tokens held in shared memory.
 template <int TT>
 __global__ void __launch_bounds__(256) router_simt_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     constexpr int KC = 256;  // columns staged per pass
     __shared__ __align__(16) float xs[KC * TT];
     const int e = threadIdx.x;
@@ -71,12 +73,11 @@ __global__ void __launch_bounds__(256) router_simt_kernel(Ctx c) {
 cudaError_t launch_router_simt(const Ctx& c, cudaStream_t st) {
     if (c.ks > 1) {
         dim3 grid((c.T + kRouterTTSmall - 1) / kRouterTTSmall, c.ks);
-        router_simt_kernel<kRouterTTSmall><<<grid, 256, 0, st>>>(c);
+        return launch_pdl(router_simt_kernel<kRouterTTSmall>, grid, dim3(256), 0, st, c);
     } else {
         dim3 grid((c.T + kRouterTT - 1) / kRouterTT, 1);
-        router_simt_kernel<kRouterTT><<<grid, 256, 0, st>>>(c);
+        return launch_pdl(router_simt_kernel<kRouterTT>, grid, dim3(256), 0, st, c);
     }
-    return cudaGetLastError();
 }
 
 __device__ __forceinline__ uint32_t bf16x2_to_half2_bits(uint32_t w, bool* range_bad) {
@@ -102,6 +103,8 @@ __device__ __forceinline__ uint32_t ord_key(float v) {
 }
 
 __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int lane = lane_id();
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= c.T) return;
@@ -233,8 +236,7 @@ __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
 }
 
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st) {
-    topk_kernel<<<(c.T + 7) / 8, 256, 0, st>>>(c, histogram ? 1 : 0);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel, dim3((c.T + 7) / 8), dim3(256), 0, st, c, histogram ? 1 : 0);
 }
 
 // ---- bucket scan + tile list (one CTA) ---------------------------------------------------------
@@ -252,6 +254,8 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 // time), the quarters are combined in shared memory, and a second pass writes every block's base
 // inside each bucket back into the histogram rows.
 __global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     __shared__ int part[4][256];
     __shared__ int cnt[264], off[264], toff[264];
     const int tid = threadIdx.x, lane = lane_id();
@@ -318,13 +322,14 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
 }
 
 cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st) {
-    bucket_scan_kernel<<<1, 1024, 0, st>>>(c);
-    return cudaGetLastError();
+    return launch_pdl(bucket_scan_kernel, dim3(1), dim3(1024), 0, st, c);
 }
 
 // ---- scatter: bucket positions and row metadata ---------------------------------------------
 
 __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ int sm[];
     int* cnt = sm;          // [E] next free row of each bucket for this CTA
     const int lane = lane_id(), warp = threadIdx.x >> 5;
@@ -387,8 +392,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
 
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st) {
     const size_t smem = sizeof(int) * (size_t)c.E;
-    scatter_kernel<<<c.nblk, 256, smem, st>>>(c);
-    return cudaGetLastError();
+    return launch_pdl(scatter_kernel, dim3(c.nblk), dim3(256), smem, st, c);
 }
 
 }  // namespace moe

@@ -33,6 +33,8 @@ constexpr int kRSmem = kROffBar + (2 * kRStages + 2) * 8 + 16 + 1024;
 
 __global__ void __launch_bounds__(kRThreads, 1)
     router_tc_kernel(Ctx c, int n_exp, const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX) {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kROffBar);
@@ -175,8 +177,7 @@ cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmW, const CUtenso
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
     if (e != cudaSuccess) return e;
     dim3 grid((c.T + kRM - 1) / kRM, kRSplit);
-    router_tc_kernel<<<grid, kRThreads, kRSmem, st>>>(c, n_exp, tmW, tmX);
-    return cudaGetLastError();
+    return launch_pdl(router_tc_kernel, grid, dim3(kRThreads), kRSmem, st, c, n_exp, tmW, tmX);
 }
 
 }  // namespace moe

@@ -72,10 +72,17 @@ extern "C" {
 /* ---- configuration flags ---------------------------------------------------------------------- */
 #define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
 #define MOE_FLAG_DECODE_UNFUSED  0x2u  /* T == 1: use the multi-kernel GEMV chain instead of the
-                                          single cooperative decode kernel */
-#define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its first load,
-                                          so the consumers' bounded waits run out and the call
-                                          reports MOE_ERR_DEVICE_TIMEOUT; nothing traps or hangs */
+                                          single fused decode kernel */
+#define MOE_FLAG_POISON_WORKSPACE 0x4u /* test aid: the handle's workspace starts filled with 0xFF
+                                          bytes (NaN floats, -1 indices) instead of zeros, except
+                                          the words the kernels count on starting at zero, so a
+                                          read of workspace no kernel wrote shows up as a wrong or
+                                          non-finite result (results are otherwise unchanged) */
+#define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its loads on
+                                          every call, and the fused batch-1 decode kernel withholds
+                                          one router result on the handle's first call, so bounded
+                                          waits run out and the call reports
+                                          MOE_ERR_DEVICE_TIMEOUT; nothing traps or hangs */
 
 typedef struct moe_handle moe_handle;
 

@@ -85,6 +85,22 @@ def test_small_shapes(shape, path):
     layer.close()
 
 
+@pytest.mark.parametrize("shape", [TINY, RAGGED], ids=lambda s: s.name)
+def test_poisoned_workspace_changes_no_result(shape):
+    """Sanitiser substitute: the workspace starts as 0xFF bytes (NaN / -1) instead of zeros, so a
+    kernel that reads workspace it did not write first would give non-finite or wrong outputs.
+    Both paths (prefill; batch-1 fused decode; multi-token GEMV decode) still match the oracle."""
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    for dec in (0, shape.T):
+        layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=dec, flags=M.MOE_FLAG_POISON_WORKSPACE)
+        _route_check(layer, ol, x, shape)
+        for T in sorted({1, 2, min(shape.T, 129), shape.T}):
+            _forward_check(layer, ol, x[:T])
+        layer.close()
+
+
 def test_tiny_intermediate_activations_match():
     """The gate/up GEMM alone: act rows in bucket order vs silu(Wg x) * (Wu x) from the oracle's
     dequantised weights (fp64), within fp16 rounding."""
@@ -321,4 +337,31 @@ def test_stalled_wait_times_out_and_the_context_stays_usable():
     stalled.close()
     layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=0)
     _forward_check(layer, ol, x)
+    layer.close()
+
+
+def test_decode_call_after_a_timed_out_one_is_correct():
+    """Batch-1 decode: with the test-only stall flag the fused kernel withholds one router result
+    on the handle's first call, so the routed units' bounded waits run out (about 1 s) and the call
+    gives up part-way, leaving partial sums in the workspace.  The very next call -- made without
+    reading the status in between -- must reset that state on the device and compute the right
+    output; the status then reports the first call's timeout once."""
+    shape = TINY
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol, T=1)
+    ref = ol.forward(x)
+    layer = _layer(w, shape, max_tokens=1, decode_max_tokens=1, flags=M.MOE_FLAG_TEST_STALL)
+    xc = x.cuda()
+    layer.forward(xc)                    # gives up part-way
+    out = layer.forward(xc)              # no status read in between
+    torch.cuda.synchronize()
+    compare(out.cpu(), ref)
+    assert layer.status() == M.MOE_ERR_DEVICE_TIMEOUT
+    assert layer.status() == M.MOE_OK
+    for _ in range(2):
+        out = layer.forward(xc)
+    torch.cuda.synchronize()
+    compare(out.cpu(), ref)
+    assert layer.status() == M.MOE_OK
     layer.close()
