@@ -362,4 +362,19 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same without the shifts, for the two nibble positions of a 16-bit half that lie inside the
+// fp16 mantissa.  Position 0 (bits 0-3 and 16-19): 1024 + q - 1024 = q.  Position 1 (bits 4-7 and
+// 20-23): OR-ed under the same exponent the half reads 1024 + 16 q, so the result is 16 q (exact).
+// One mask-and-or (LOP3) and one subtraction per pair.
+__device__ __forceinline__ __half2 nibble_pair_pos0(uint32_t word) {
+    uint32_t v = (word & 0x000F000Fu) | 0x64006400u;
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    return __hsub2(h, __half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+}
+__device__ __forceinline__ __half2 nibble_pair_pos1(uint32_t word) {
+    uint32_t v = (word & 0x00F000F0u) | 0x64006400u;
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    return __hsub2(h, __half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+}
+
 }  // namespace moe

@@ -68,8 +68,15 @@ struct GemmCfg {
     static constexpr int kBN = CTAS == 1 ? 256 : 128;   // token columns per tile (= UMMA N)
     static constexpr int kEpiWarps = 8 / CTAS;
     static constexpr int kTransformWarps = 8 / CTAS;
-    static constexpr int kEpiWarp0 = 2 + kTransformWarps;
-    static constexpr int kThreads = 32 * (2 + kTransformWarps + kEpiWarps);
+    // Warp roles, placed by scheduler (warp % 4): the MMA-issuing warp 1 must not share its
+    // scheduler with the busy transform warps (measured: a tcgen05.mma issue took ~110 cycles
+    // when it did, against ~45 alone), so the epilogue warps (idle between tiles) take warps
+    // 2 .. 2 + kEpiWarps - 1 and the transform warps the following warps whose index is not 1
+    // mod 4; those left over stay idle.
+    static constexpr int kEpiWarp0 = 2;
+    static constexpr int kXWarp0 = 2 + kEpiWarps;   // first transform-candidate warp
+    static constexpr int kXCand = kTransformWarps + (kTransformWarps - 1) / 3;   // skipping every 4th
+    static constexpr int kThreads = 32 * (kXWarp0 + kXCand);
     static constexpr int kTmemCols = 512 / CTAS;
     static constexpr int kAccCols = kBN;
     static constexpr int kWB = CTAS == 1 ? 4 : 2;   // weight blocks per bulk copy
@@ -254,12 +261,12 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                     if (!mbar_wait(&afull[as], aph, abort_flag, c.status)) goto mma_done;
                     if (!mbar_wait(&bfull[bs], bph, abort_flag, c.status)) goto mma_done;
                     tc_fence_after();
-                    const uint32_t a_addr = a0 + as * kATileBytes, b_addr = b0 + bs * kBTileBytes;
+                    // descriptors of the stage once; the kk-th 16-column slice starts 32 bytes on,
+                    // i.e. +2 in the start-address field (no carry: shared addresses < 256 KB)
+                    const uint64_t ad = sdesc_sw128(a0 + as * kATileBytes), bd = sdesc_sw128(b0 + bs * kBTileBytes);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        mma_ss(d_tmem, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
-                               (kc | kk) != 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kc | kk) != 0 ? 1u : 0u);
                     issued = true;
                     tc_commit(&aempty[as]);
                     tc_commit(&bempty[bs]);
@@ -275,17 +282,20 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 mbar_drain(drainbar, 0);
             }
         }
-    } else if (warp < kEpiWarp0) {
+    } else if (warp >= K::kXWarp0) {
         // ------------------------------------------------------------------ transform
         // thread = (weight row, half of the 64 columns; both halves when there are 4 transform
         // warps); the fp16 pairs of 16-byte chunk ch of row r go to r*128 + ((ch ^ (r & 7)) * 16),
         // the 128-byte swizzle the MMA descriptor expects.
-        const int tt = threadIdx.x - 64;        // 0 .. 32 * kTransformWarps - 1
+        const int wx = warp - K::kXWarp0;      // candidates: every warp not on scheduler 1
+        const int ti = wx - (wx >> 2);          // transform warp index (when wx % 4 != 3)
+        const bool active = (wx & 3) != 3 && ti < kTransformWarps;
+        const int tt = ti * 32 + lane;          // 0 .. 32 * kTransformWarps - 1
         const int row = tt & 127;
         const uint32_t sw = (uint32_t)(row & 7);
         int ws = 0, as = 0;
         uint32_t wph = 0, aph = 0;
-        for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+        for (int tau = active ? (int)blockIdx.x : total; tau < total; tau += gridDim.x) {
             const int4 tile = c.tiles1[tau / MT];
             if (!tile_ok(tile, c, kBN)) continue;
             for (int kc = 0; kc < KS; ++kc) {
@@ -304,17 +314,21 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)),
                                            __ushort_as_half((unsigned short)(sb >> 16)));
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                // codes of nibble position 1 (bits 4-7 of each 16-bit half) are read in place as
+                // 16 q, so their scale is s / 16 (exact in fp16 for |s| >= 2^-13)
+                const __half2 s2_16 = __hmul2(s2, __half2(__float2half(0.0625f), __float2half(0.0625f)));
                 uint8_t* arow = asm_ + as * kATileBytes + row * 128;
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    uint32_t r[4];
-#pragma unroll
-                    for (int sft = 0; sft < 4; ++sft) {
-                        const __half2 v = __hfma2(codes_to_half2(words[w], sft), s2, b2);
-                        r[sft] = *reinterpret_cast<const uint32_t*>(&v);
-                    }
+                    const uint32_t lo = words[w], hi = words[w] >> 8;   // positions 0,1 | 2,3 (one shift)
+                    const __half2 v0 = __hfma2(nibble_pair_pos0(lo), s2, b2);
+                    const __half2 v1 = __hfma2(nibble_pair_pos1(lo), s2_16, b2);
+                    const __half2 v2 = __hfma2(nibble_pair_pos0(hi), s2, b2);
+                    const __half2 v3 = __hfma2(nibble_pair_pos1(hi), s2_16, b2);
                     const uint32_t ch = (uint32_t)(4 * half + w);
-                    *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(r[0], r[1], r[2], r[3]);
+                    *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) =
+                        make_uint4(*reinterpret_cast<const uint32_t*>(&v0), *reinterpret_cast<const uint32_t*>(&v1),
+                                   *reinterpret_cast<const uint32_t*>(&v2), *reinterpret_cast<const uint32_t*>(&v3));
                 }
                 }
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core

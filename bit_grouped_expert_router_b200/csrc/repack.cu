@@ -7,8 +7,9 @@
 //             pair them with one shuffle (SwiGLU without a trip through shared memory).
 //   down    : (H/128) m-tiles x (I/64) k-steps; block row l is output row 128*mt + l.
 // Group g < E is routed expert g, group E the shared expert.  Scales and biases are converted
-// from bf16 to fp16 (round to nearest even); any value that is not exactly representable in fp16
-// raises a flag that moe_create reports in its message (the weights stay usable).
+// from bf16 to fp16 (round to nearest even); any value that is not exactly representable in fp16,
+// and any nonzero scale below 2^-13 in magnitude (the dequantisation also uses s / 16), raises a
+// flag that moe_create reports in its message (the weights stay usable).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -74,6 +75,10 @@ __global__ void __launch_bounds__(256) repack_kernel(RepackArgs a) {
         const uint16_t* b2 = shared ? a.bs[m2] : a.b[m2] + (size_t)g * mat_groups;
         const size_t gi = (size_t)row2 * (cols / 64) + c;
         const uint32_t sh = bf16_to_fp16_bits(s2[gi], a.inexact);
+        {   // the tensor-core dequantisation also uses s / 16, exact in fp16 only for |s| >= 2^-13
+            const float sf = fabsf(__half2float(__ushort_as_half((unsigned short)sh)));
+            if (sf != 0.f && sf < 0.0001220703125f) atomicOr(a.inexact, 1u);
+        }
         const uint32_t bh = bf16_to_fp16_bits(b2[gi], a.inexact);
         *reinterpret_cast<uint32_t*>(blk + kBlockCodeBytes + 4 * r2) = sh | (bh << 16);
     }

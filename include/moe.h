@@ -128,7 +128,9 @@ typedef struct {
  * so the caller may free its weight buffers as soon as it returns.  On success *out receives the
  * handle.  Allocates device memory (the only entry point that does).  Scales/biases that are not
  * exactly representable in fp16 are rounded to nearest (the layer still works; the tensor-core
- * path computes in fp16).  Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+ * path computes in fp16), and nonzero scales below 2^-13 in magnitude are not reproduced exactly
+ * by the tensor-core dequantisation (it also uses s / 16).  Errors: INVALID_ARG,
+ * UNSUPPORTED_DEVICE, CUDA. */
 MOE_API int moe_create(const moe_config *cfg, const moe_weights *w, int device, void *stream,
                moe_handle **out);
 
