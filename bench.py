@@ -60,6 +60,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the prefill512 / prefill4k_zipf fractions")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle sample time")
+    ap.add_argument("--ablations", action="store_true",
+                    help="also time the pages' two prefill ablations (host-synchronised routing, fp16 "
+                         "weights dequantised once into HBM) against the product path")
     return ap.parse_args()
 
 
@@ -161,7 +164,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------------------- stacks
-def build_stack(shape, n_layers, max_tokens, decode_max_tokens, keep_host_layer0=False):
+def build_stack(shape, n_layers, max_tokens, decode_max_tokens, keep_host_layer0=False, flags=0):
     import torch
     from bit_grouped_expert_router_b200 import _lib as M
     from bit_grouped_expert_router_b200 import synth
@@ -170,7 +173,8 @@ def build_stack(shape, n_layers, max_tokens, decode_max_tokens, keep_host_layer0
         w = synth.make_layer(shape, l, device="cuda")
         if l == 0 and keep_host_layer0:
             host0 = {k: (v.cpu() if v is not None else None) for k, v in w.items()}
-        layers.append(M.Layer.from_shape(w, shape, max_tokens=max_tokens, decode_max_tokens=decode_max_tokens))
+        layers.append(M.Layer.from_shape(w, shape, max_tokens=max_tokens, decode_max_tokens=decode_max_tokens,
+                                         flags=flags))
         del w
     torch.cuda.synchronize()
     return layers, host0
@@ -472,6 +476,46 @@ def run_configs(args, dist, peaks, peak_src):
     return out
 
 
+def run_ablations(args, dist):
+    """The pages' prefill levers, each against the product path on the same 4 layers (eager calls,
+    CUDA events): GPU-resident routing vs a host round trip between routing and the expert GEMMs
+    (MOE_FLAG_HOST_SYNC_ROUTING), and 4-bit weights rebuilt inside the grouped GEMM vs fp16
+    weights dequantised once into HBM (MOE_FLAG_DEQUANT_TO_HBM).  us per layer call."""
+    import torch
+    from bit_grouped_expert_router_b200 import _lib as M
+    from bit_grouped_expert_router_b200 import synth
+    out = {}
+    variants = (("product", 0), ("host_sync_routing", M.MOE_FLAG_HOST_SYNC_ROUTING),
+                ("fp16_weights_in_hbm", M.MOE_FLAG_DEQUANT_TO_HBM))
+    for name in ("prefill16k_zipf", "prefill512"):
+        shape = synth.WORKLOADS[name]
+        n = 4
+        xs = [synth.make_x(shape, l, 0, device="cuda") for l in range(n)]
+        row = {}
+        for vname, flags in variants:
+            layers, _ = build_stack(shape, n, shape.T, 16, flags=flags)
+
+            def step():
+                for l in range(n):
+                    layers[l].forward(xs[l])
+
+            reps = max(args.steps, 5)
+            row[vname] = round(timed(step, reps, 3, dist) * 1000.0 / n, 2)
+            prof = profile_pass(layers, step, reps)
+            row[vname + "_gemm_us"] = round(prof["gemm_gateup"]["avg_us"] + prof["gemm_down"]["avg_us"], 2)
+            for L in layers:
+                assert L.status() == 0
+                L.close()
+            del layers
+            torch.cuda.empty_cache()
+        for vname, _ in variants[1:]:
+            row[vname + "_vs_product"] = round(row[vname] / row["product"], 4)
+        out[name] = row
+        del xs
+    out["unit"] = "us per layer call (eager), and the two grouped GEMMs' kernel time"
+    return out
+
+
 def run_decode(args, dist, peaks, peak_src):
     import torch
     from bit_grouped_expert_router_b200 import synth
@@ -681,6 +725,8 @@ def main():
             line["decode"] = d
         if not args.no_configs and dist.world == 1:
             line["other_configs"] = run_configs(args, dist, peaks, peak_src)
+        if args.ablations and dist.world == 1:
+            line["ablations"] = run_ablations(args, dist)
         line["config"] = prefill_config(args, shape, r["n_layers"])
     base = {"n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16", "data": "synthetic (seeded random-init weights and activations)"}

@@ -27,6 +27,8 @@ MOE_ERR_RANGE = 7
 MOE_FLAG_ROUTER_SIMT = 0x1
 MOE_FLAG_DECODE_UNFUSED = 0x2
 MOE_FLAG_POISON_WORKSPACE = 0x4
+MOE_FLAG_HOST_SYNC_ROUTING = 0x8
+MOE_FLAG_DEQUANT_TO_HBM = 0x10
 MOE_FLAG_TEST_STALL = 0x100
 
 _ERR_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DEVICE", 3: "TOO_LARGE", 4: "CUDA",

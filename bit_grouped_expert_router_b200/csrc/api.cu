@@ -174,7 +174,7 @@ int validate_config(const moe_config* c) {
     if ((c->decode_max_tokens >= 2 || (c->flags & MOE_FLAG_DECODE_UNFUSED)) && c->top_k + c->has_shared > 16)
         return fail(MOE_ERR_INVALID_ARG, "the multi-kernel decode path supports top_k + has_shared <= 16");
     if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_DECODE_UNFUSED | MOE_FLAG_POISON_WORKSPACE |
-                               MOE_FLAG_TEST_STALL))
+                               MOE_FLAG_HOST_SYNC_ROUTING | MOE_FLAG_DEQUANT_TO_HBM | MOE_FLAG_TEST_STALL))
         return fail(MOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
     return MOE_OK;
 }
@@ -238,6 +238,10 @@ struct moe_handle {
     uint16_t* wsplit = nullptr;
     cudaStream_t last_stream = nullptr;
     bool inexact_scales = false;
+    // MOE_FLAG_DEQUANT_TO_HBM: the layer's weights dequantised once to fp16 rows in HBM, and
+    // their tensor maps (box 64 columns x 128 rows), for the grouped-GEMM ablation variant
+    __half* w16 = nullptr;
+    CUtensorMap amap_gu{}, amap_dn{};
     // batch-1 decode: the fused kernel's geometry, when the shape and the device allow it
     bool fused_ok = false;
     DecodeGeom dgeom{};
@@ -326,7 +330,10 @@ const char* moe_last_error(void) { return g_last_error.c_str(); }
 size_t moe_device_bytes(const moe_config* cfg) {
     if (validate_config(cfg) != MOE_OK) return 0;
     const Layout L = make_layout(*cfg);
-    return L.weights_bytes + L.ws_bytes;
+    size_t extra = 0;
+    if (cfg->flags & MOE_FLAG_DEQUANT_TO_HBM)
+        extra = sizeof(__half) * ((size_t)L.G * 2 * L.I * L.H + (size_t)L.G * L.H * L.I);
+    return L.weights_bytes + L.ws_bytes + extra;
 }
 
 int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* stream, moe_handle** out) {
@@ -366,6 +373,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     h->num_sms = prop.multiProcessorCount;
     const Layout& L = h->L;
     auto cleanup = [&](int code) {
+        if (h->w16) cudaFree(h->w16);
         if (h->wbuf) cudaFree(h->wbuf);
         if (h->ws) cudaFree(h->ws);
         delete h;
@@ -495,6 +503,19 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     if (rc == MOE_OK)
         rc = encode_rows_map(&h->tm_wsplit, wsplit, L.Epad, 2 * L.H, router_n_exp(L), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc != MOE_OK) return cleanup(rc);
+    if (cfg->flags & MOE_FLAG_DEQUANT_TO_HBM) {
+        const size_t rows_gu = (size_t)L.G * (L.I / 64) * 128, rows_dn = (size_t)L.G * (L.H / 128) * 128;
+        e = cudaMalloc(&h->w16, sizeof(__half) * (rows_gu * L.H + rows_dn * L.I));
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMalloc(fp16 weights): %s", cudaGetErrorString(e)));
+        __half* w16_dn = h->w16 + rows_gu * L.H;
+        e = launch_dequant_rows(w_gu, L.G, L.I / 64, L.H / 64, h->w16, st);
+        if (e == cudaSuccess) e = launch_dequant_rows(w_dn, L.G, L.H / 128, L.I / 64, w16_dn, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "fp16 weights: %s", cudaGetErrorString(e)));
+        rc = encode_rows_map(&h->amap_gu, h->w16, (int)rows_gu, L.H, 128);
+        if (rc == MOE_OK) rc = encode_rows_map(&h->amap_dn, w16_dn, (int)rows_dn, L.I, 128);
+        if (rc != MOE_OK) return cleanup(rc);
+    }
     h->last_stream = st;
     *out = h;
     return MOE_OK;
@@ -525,9 +546,25 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     } else {
         MOE_LAUNCH("moe.gather_rows", launch_gather_rows(c, h->num_sms, st));
         pf.mark(10);
-        MOE_LAUNCH("moe.gemm_gateup", launch_gemm_gateup(c, h->maps_gu, h->num_sms, st));
+        int sms_gu = h->num_sms, sms_dn = h->num_sms;
+        if (h->cfg.flags & MOE_FLAG_HOST_SYNC_ROUTING) {
+            // ablation of GPU-resident routing: the host waits for the routing kernels, reads the
+            // tile count back and sizes the grouped GEMMs' grids from it (same results)
+            int nt = 0;
+            {
+                NvtxRange r("moe.host_sync_routing");
+                CUDA_TRY(cudaMemcpyAsync(&nt, c.ntiles, sizeof(int), cudaMemcpyDeviceToHost, st));
+                CUDA_TRY(cudaStreamSynchronize(st));
+            }
+            const int per_cta = c.tile_rows == 128 ? 2 : 1;   // CTAs per SM of the launch shape
+            auto sms_for = [&](int tasks) { return std::max(1, std::min(h->num_sms, (tasks + per_cta - 1) / per_cta)); };
+            sms_gu = sms_for(nt * (h->L.I / 64));
+            sms_dn = sms_for(nt * (h->L.H / 128));
+        }
+        const bool a16 = h->w16 != nullptr;
+        MOE_LAUNCH("moe.gemm_gateup", launch_gemm_gateup(c, h->maps_gu, a16 ? &h->amap_gu : nullptr, sms_gu, st));
         pf.mark(4);
-        MOE_LAUNCH("moe.gemm_down", launch_gemm_down(c, h->maps_dn, h->num_sms, st));
+        MOE_LAUNCH("moe.gemm_down", launch_gemm_down(c, h->maps_dn, a16 ? &h->amap_dn : nullptr, sms_dn, st));
         pf.mark(5);
         MOE_LAUNCH("moe.finalize", launch_finalize(c, st));
         pf.mark(6);
@@ -669,6 +706,7 @@ void moe_destroy(moe_handle* h) {
             for (int i = 0; i < kProfCalls * kProfEvents; ++i) cudaEventDestroy(h->prof_ev[i]);
             delete[] h->prof_ev;
         }
+        if (h->w16) cudaFree(h->w16);
         if (h->wbuf) cudaFree(h->wbuf);
         if (h->ws) cudaFree(h->ws);
     }

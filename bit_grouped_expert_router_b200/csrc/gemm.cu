@@ -112,9 +112,12 @@ __device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c, int bn) {
     return t.x >= 0 && t.x < c.G && t.y >= 0 && t.z > 0 && t.z <= bn && t.y + t.z <= c.rows_cap;
 }
 
-template <bool GATEUP, int CTAS>
+// AHBM: the ablation variant that reads A as fp16 weights dequantised once into HBM (one 2-D TMA
+// tile per k-step, box 64 columns x 128 rows, the same 128-byte swizzle the transform writes)
+// instead of rebuilding it from the 4-bit blocks in shared memory; the transform warps idle.
+template <bool GATEUP, int CTAS, bool AHBM>
 __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
-    grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps) {
+    grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps, const __grid_constant__ CUtensorMap amap) {
     griddep_wait();
     griddep_launch_dependents();
     using K = GemmCfg<CTAS>;
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             mbar_init(&bempty[s], 1);
         }
         for (int s = 0; s < kAS; ++s) {
-            mbar_init(&afull[s], kTransformWarps);
+            mbar_init(&afull[s], AHBM ? 1 : kTransformWarps);
             mbar_init(&aempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         fence_mbar_init();
         for (int i = 0; i < 2; ++i)
             for (int j = 0; j < 3; ++j) prefetch_tmap(&maps.m[i][j]);
+        if (AHBM) prefetch_tmap(&amap);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -189,9 +193,9 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         // Lane 0 waits for ring slots and issues the copies (the rest of the warp follows along).
         if (!(c.flags & 0x100u)) {
             const int shared_base = (GATEUP && c.has_shared) ? c.offsets[c.E] : 0;
-            uint32_t wit = 0, bit = 0;
-            int ws = 0, bs = 0;
-            uint32_t wph = 0, bph = 0;
+            uint32_t wit = 0, bit = 0, ait = 0;
+            int ws = 0, bs = 0, as = 0;
+            uint32_t wph = 0, bph = 0, aph = 0;
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
                 const int mt = tau % MT;
@@ -205,8 +209,17 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 const uint8_t* wsrc = wbase + ((size_t)tile.x * MT + mt) * KS * kBlockBytes;
                 for (int kc = 0; kc < KS; ++kc) {
                     int ok = 1;
-                    if (lane == 0) {
-                        if (kc % kWB == 0) {
+                    if (lane == 0 && AHBM) {   // the fp16 A tile of this k-step from HBM
+                        ok = mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status) ? 1 : 0;
+                        if (ok) {
+                            mbar_arrive_expect_tx(&afull[as], (uint32_t)kATileBytes);
+                            tma_load_2d(asm_ + as * kATileBytes, &amap, kc * 64, (tile.x * MT + mt) * 128, &afull[as]);
+                            ++ait;
+                            if (++as == kAS) { as = 0; aph ^= 1u; }
+                        }
+                    }
+                    if (lane == 0 && ok) {
+                        if (!AHBM && kc % kWB == 0) {
                             const int nb = min(kWB, KS - kc);
                             ok = mbar_wait(&wempty[ws], wph ^ 1u, abort_flag, c.status) ? 1 : 0;
                             if (ok) {
@@ -236,6 +249,8 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                     mbar_drain(&wfull[i % kWS], (i / kWS) & 1u);
                 for (uint32_t i = bit > (uint32_t)kBS ? bit - kBS : 0u; i < bit; ++i)
                     mbar_drain(&bfull[i % kBS], (i / kBS) & 1u);
+                for (uint32_t i = ait > (uint32_t)kAS ? ait - kAS : 0u; i < ait; ++i)
+                    mbar_drain(&afull[i % kAS], (i / kAS) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -289,7 +304,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         // the 128-byte swizzle the MMA descriptor expects.
         const int wx = warp - K::kXWarp0;      // candidates: every warp not on scheduler 1
         const int ti = wx - (wx >> 2);          // transform warp index (when wx % 4 != 3)
-        const bool active = (wx & 3) != 3 && ti < kTransformWarps;
+        const bool active = !AHBM && (wx & 3) != 3 && ti < kTransformWarps;
         const int tt = ti * 32 + lane;          // 0 .. 32 * kTransformWarps - 1
         const int row = tt & 127;
         const uint32_t sw = (uint32_t)(row & 7);
@@ -475,13 +490,26 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(Ctx c) {
 
 namespace {
 
-template <bool GATEUP, int CTAS>
-cudaError_t launch_grouped(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
+template <bool GATEUP, int CTAS, bool AHBM>
+cudaError_t launch_grouped(const Ctx& c, const TokenMaps& maps, const CUtensorMap& amap, int num_sms, cudaStream_t st) {
     using K = GemmCfg<CTAS>;
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, CTAS>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, CTAS, AHBM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmemBytes);
     if (e != cudaSuccess) return e;
-    return launch_pdl(grouped_gemm_kernel<GATEUP, CTAS>, dim3(num_sms * CTAS), dim3(K::kThreads), K::kSmemBytes, st, c, maps);
+    return launch_pdl(grouped_gemm_kernel<GATEUP, CTAS, AHBM>, dim3(num_sms * CTAS), dim3(K::kThreads), K::kSmemBytes,
+                      st, c, maps, amap);
+}
+
+template <bool GATEUP>
+cudaError_t launch_shape(const Ctx& c, const TokenMaps& maps, const CUtensorMap* amap, int num_sms, cudaStream_t st) {
+    static const CUtensorMap kNoMap = {};
+    if (c.tile_rows == GemmCfg<2>::kBN)
+        return amap ? launch_grouped<GATEUP, 2, true>(c, maps, *amap, num_sms, st)
+                    : launch_grouped<GATEUP, 2, false>(c, maps, kNoMap, num_sms, st);
+    if (c.tile_rows == GemmCfg<1>::kBN)
+        return amap ? launch_grouped<GATEUP, 1, true>(c, maps, *amap, num_sms, st)
+                    : launch_grouped<GATEUP, 1, false>(c, maps, kNoMap, num_sms, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -494,17 +522,16 @@ cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st) {
     return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, c);
 }
 
-// The tile list (built for c.tile_rows rows per tile) selects the launch shape.
-cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
-    if (c.tile_rows == GemmCfg<2>::kBN) return launch_grouped<true, 2>(c, maps, num_sms, st);
-    if (c.tile_rows == GemmCfg<1>::kBN) return launch_grouped<true, 1>(c, maps, num_sms, st);
-    return cudaErrorInvalidValue;
+// The tile list (built for c.tile_rows rows per tile) selects the launch shape; amap (non-NULL)
+// selects the fp16-weights-in-HBM ablation variant.
+cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, const CUtensorMap* amap, int num_sms,
+                               cudaStream_t st) {
+    return launch_shape<true>(c, maps, amap, num_sms, st);
 }
 
-cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st) {
-    if (c.tile_rows == GemmCfg<2>::kBN) return launch_grouped<false, 2>(c, maps, num_sms, st);
-    if (c.tile_rows == GemmCfg<1>::kBN) return launch_grouped<false, 1>(c, maps, num_sms, st);
-    return cudaErrorInvalidValue;
+cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, const CUtensorMap* amap, int num_sms,
+                             cudaStream_t st) {
+    return launch_shape<false>(c, maps, amap, num_sms, st);
 }
 
 // out[t][h] = bf16(acc[t][h]), round to nearest even; 8 elements per thread per step.

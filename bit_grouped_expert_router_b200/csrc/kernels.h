@@ -125,8 +125,17 @@ struct TokenMaps {
 
 // prefill grouped GEMMs
 cudaError_t launch_gather_rows(const Ctx& c, int num_sms, cudaStream_t st);
-cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st);
-cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, int num_sms, cudaStream_t st);
+// amap: NULL for the in-GEMM 4-bit dequantisation; else the tensor map of the layer's weights
+// dequantised once to fp16 in HBM (the ablation variant, box 64 columns x 128 rows)
+cudaError_t launch_gemm_gateup(const Ctx& c, const TokenMaps& maps, const CUtensorMap* amap, int num_sms,
+                               cudaStream_t st);
+cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, const CUtensorMap* amap, int num_sms,
+                             cudaStream_t st);
+// Writes the layer's repacked 4-bit blocks of one matrix kind as fp16 rows: dst[(g*MT + mt)*128 + l]
+// [64*kc + j] = the weight the grouped GEMM's transform would put in row l, column j of block
+// (g, mt, kc) (the ablation's weights in HBM).
+cudaError_t launch_dequant_rows(const uint8_t* blocks, int groups, int m_tiles, int k_steps, __half* dst,
+                                cudaStream_t st);
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st);
 // Token rows per grouped-GEMM tile for a call of T tokens: 128 (two CTAs per SM) when the
 // routed experts average at most 64 tokens (T * k <= 64 * E), else 256 (one CTA per SM).

@@ -112,4 +112,36 @@ cudaError_t launch_router_prep(const float* router, const float* bias, const flo
     return cudaGetLastError();
 }
 
+// One block (g, mt, kc) per CTA of 256 threads; thread = (row, column half).  The same fp16
+// arithmetic as the grouped GEMM's transform (exact for this format).
+__global__ void __launch_bounds__(256) dequant_rows_kernel(const uint8_t* __restrict__ blocks, int m_tiles,
+                                                           int k_steps, __half* __restrict__ dst) {
+    const int kc = blockIdx.x, mt = blockIdx.y, g = blockIdx.z;
+    const int row = threadIdx.x & 127, half = threadIdx.x >> 7;
+    const uint8_t* blk = blocks + (((size_t)g * m_tiles + mt) * k_steps + kc) * kBlockBytes;
+    const uint4 cw = *reinterpret_cast<const uint4*>(blk + half * 2048 + row * 16);
+    const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+    const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)), __ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+    const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)), __ushort_as_half((unsigned short)(sb >> 16)));
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+    uint32_t out[16];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int sft = 0; sft < 4; ++sft) {   // columns 8w + 2 sft, +1 of this half
+            const __half2 v = __hfma2(codes_to_half2(words[w], sft), s2, b2);
+            out[4 * w + sft] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+    uint4* d = reinterpret_cast<uint4*>(dst + (((size_t)g * m_tiles + mt) * 128 + row) * (size_t)(64 * k_steps) +
+                                        64 * kc + 32 * half);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+}
+
+cudaError_t launch_dequant_rows(const uint8_t* blocks, int groups, int m_tiles, int k_steps, __half* dst,
+                                cudaStream_t st) {
+    dequant_rows_kernel<<<dim3(k_steps, m_tiles, groups), 256, 0, st>>>(blocks, m_tiles, k_steps, dst);
+    return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -78,6 +78,17 @@ extern "C" {
                                           the words the kernels count on starting at zero, so a
                                           read of workspace no kernel wrote shows up as a wrong or
                                           non-finite result (results are otherwise unchanged) */
+#define MOE_FLAG_HOST_SYNC_ROUTING 0x8u /* ablation of GPU-resident routing: on the prefill path
+                                          the host waits for the routing kernels and reads the tile
+                                          count back before it launches the grouped GEMMs (grids
+                                          sized from it); same results, one host round trip per
+                                          call, so moe_forward synchronises its stream and cannot
+                                          be captured in a CUDA graph */
+#define MOE_FLAG_DEQUANT_TO_HBM  0x10u /* ablation of the in-GEMM 4-bit reconstruction: moe_create
+                                          also writes the layer's weights dequantised to fp16 in
+                                          the handle's memory (4x the bytes of the packed codes),
+                                          and the prefill grouped GEMMs load those instead of
+                                          rebuilding each tile from the 4-bit blocks (same results) */
 #define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its loads on
                                           every call, and the fused batch-1 decode kernel withholds
                                           one router result on the handle's first call, so bounded

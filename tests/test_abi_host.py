@@ -45,7 +45,7 @@ def test_device_bytes_counts_the_repacked_layer(lib):
 
 @pytest.mark.parametrize("bad", [dict(group=32), dict(H=200), dict(I=96), dict(E=0), dict(E=300),
                                  dict(k=0), dict(k=33, E=64), dict(k=9, E=8), dict(max_tokens=0),
-                                 dict(decode_max_tokens=-1), dict(decode_max_tokens=65536), dict(flags=0x8), dict(flags=0x200),
+                                 dict(decode_max_tokens=-1), dict(decode_max_tokens=65536), dict(flags=0x40), dict(flags=0x200),
                                  dict(k=16, decode_max_tokens=2)])
 def test_invalid_config_is_rejected_before_any_cuda_call(lib, bad):
     cfg = _cfg(**bad)

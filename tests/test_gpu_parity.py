@@ -101,6 +101,31 @@ def test_poisoned_workspace_changes_no_result(shape):
         layer.close()
 
 
+@pytest.mark.parametrize("shape", [TINY, RAGGED], ids=lambda s: s.name)
+def test_host_synchronised_routing_ablation_changes_no_result(shape):
+    """The ablation flag only moves a host round trip between routing and the grouped GEMMs."""
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=0, flags=M.MOE_FLAG_HOST_SYNC_ROUTING)
+    for T in sorted({2, min(shape.T, 129), shape.T}):
+        _forward_check(layer, ol, x[:T])
+    layer.close()
+
+
+@pytest.mark.parametrize("shape", [TINY, RAGGED], ids=lambda s: s.name)
+def test_fp16_weights_in_hbm_ablation_matches_the_oracle(shape):
+    """The ablation variant (A tiles dequantised once to fp16 in HBM, loaded by TMA) computes the
+    same layer: both grouped-GEMM launch shapes (T * k below and above 64 * E)."""
+    w = synth.make_layer(shape)
+    ol = oracle.OracleLayer.from_shape(w, shape)
+    x = gapped_x(shape, ol)
+    layer = _layer(w, shape, max_tokens=shape.T, decode_max_tokens=0, flags=M.MOE_FLAG_DEQUANT_TO_HBM)
+    for T in sorted({2, min(shape.T, 129), shape.T}):
+        _forward_check(layer, ol, x[:T])
+    layer.close()
+
+
 def test_tiny_intermediate_activations_match():
     """The gate/up GEMM alone: act rows in bucket order vs silu(Wg x) * (Wu x) from the oracle's
     dequantised weights (fp64), within fp16 rounding."""
