@@ -71,8 +71,9 @@ extern "C" {
 
 /* ---- configuration flags ---------------------------------------------------------------------- */
 #define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
-#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* T == 1: use the multi-kernel GEMV chain instead of the
-                                          single fused decode kernel */
+#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* decode calls of T <= 4 tokens: use the multi-kernel
+                                          GEMV chain instead of the fused single-token kernel
+                                          (launched once per token) */
 #define MOE_FLAG_POISON_WORKSPACE 0x4u /* test aid: the handle's workspace starts filled with 0xFF
                                           bytes (NaN floats, -1 indices) instead of zeros, except
                                           the words the kernels count on starting at zero, so a
