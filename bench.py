@@ -556,7 +556,8 @@ def run_decode(args, dist, peaks, peak_src):
         a = b / (us_layer * 1e-6) / 1e9
         roof = {"bound": "hbm", "kernel": "decode_fused_kernel (one launch per layer, timed in the graph)",
                 "achieved": round(a, 1), "peak": hbm, "unit": "GB/s", "frac": round(a / hbm, 4),
-                "traffic": None, "bytes_per_token": b, "peak_source": f"{peak_src} hbm_gbs"}
+                "traffic": profiled_traffic("decode_fused", "decode_fused_decode_2layers.md", "decode_fused.cu"),
+                "bytes_per_token": b, "peak_source": f"{peak_src} hbm_gbs"}
     elif "gemv_gateup" in prof and "gemv_down" in prof:
         b_gu = nexp * (shape.I // 64) * (shape.H // 64) * 4608 + shape.H * 2
         b_dn = nexp * (shape.H // 128) * (shape.I // 64) * 4608 + shape.H * 2
@@ -584,13 +585,13 @@ def run_decode(args, dist, peaks, peak_src):
 
 
 # ------------------------------------------------------------------------------------ ncu traffic
-def kernel_code_hash():
-    """sha256 (16 hex digits) of the grouped-GEMM kernel code: csrc/gemm.cu, common.cuh and
-    kernels.h with comments and whitespace removed, concatenated (comment edits keep the hash)."""
+def kernel_code_hash(main="gemm.cu"):
+    """sha256 (16 hex digits) of a kernel's code: csrc/<main>, common.cuh and kernels.h with
+    comments and whitespace removed, concatenated (comment edits keep the hash)."""
     import hashlib
     here = os.path.dirname(os.path.abspath(__file__))
     h = hashlib.sha256()
-    for f in ("gemm.cu", "common.cuh", "kernels.h"):
+    for f in (main, "common.cuh", "kernels.h"):
         with open(os.path.join(here, "bit_grouped_expert_router_b200", "csrc", f)) as fh:
             src = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
@@ -598,17 +599,17 @@ def kernel_code_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel):
+def profiled_traffic(kernel, summary="grouped_gemm_prefill16k_zipf_1layer.md", main="gemm.cu"):
     """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary, or None when
     the kernel code changed since that capture (the summary records kernel_code_hash())."""
     here = os.path.dirname(os.path.abspath(__file__))
-    prof = os.path.join(here, "profiles", "grouped_gemm_prefill16k_zipf_1layer.md")
+    prof = os.path.join(here, "profiles", summary)
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
     m = re.search(r"kernel_sources_sha256_16: ([0-9a-f]{16})", text)
     t = re.search(r"traffic_bytes_per_launch %s: (\d+)" % re.escape(kernel), text)
-    if not m or not t or m.group(1) != kernel_code_hash():
+    if not m or not t or m.group(1) != kernel_code_hash(main):
         return None
     return int(t.group(1))
 
