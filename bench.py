@@ -222,6 +222,39 @@ def gemm_flops(shape):
     return 2.0 * rows * 2 * shape.I * shape.H, 2.0 * rows * shape.I * shape.H
 
 
+def tile_stats(layers, xs, shape, prof, clk):
+    """Tile fill and executed k-steps of the grouped GEMMs over every (layer, chunk) call of a step,
+    from the library's own routing (moe_route's bucket offsets).  The tile height follows the
+    library's launch-shape rule (256-token tiles when T*k > 64*E, else 128).  fill = bucket rows /
+    (tiles x tile height); a k-step is one 64-deep slice of the contraction for one 128-row
+    m-tile, so cycles_per_kstep = launch time x SM clock x SMs / k-steps."""
+    import torch
+    tile_rows = 256 if shape.T * shape.k > 64 * shape.E else 128
+    tiles, rows, calls = 0, 0, 0
+    for l, L in enumerate(layers):
+        for x in xs[l]:
+            off = L.route(x)["offsets"].to(torch.int64)
+            cnt = off[1:] - off[:-1]
+            tiles += int(((cnt + tile_rows - 1) // tile_rows).sum())
+            rows += int(cnt.sum())
+            if shape.has_shared:
+                tiles += (shape.T + tile_rows - 1) // tile_rows
+                rows += shape.T
+            calls += 1
+    tiles_per_call = tiles / calls
+    ks_gu = tiles_per_call * (2 * shape.I // 128) * (shape.H // 64)
+    ks_dn = tiles_per_call * (shape.H // 128) * (shape.I // 64)
+    out = {"tile_rows": tile_rows, "tiles_per_launch": round(tiles_per_call, 1),
+           "tile_fill": round(rows / (tiles * tile_rows), 4),
+           "ksteps_per_launch": {"gemm_gateup": round(ks_gu), "gemm_down": round(ks_dn)}}
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mhz = (clk or {}).get("sm_mhz")
+    if mhz:
+        out["cycles_per_kstep"] = {
+            k: round(prof[k]["avg_us"] * mhz * sms / n) for k, n in (("gemm_gateup", ks_gu), ("gemm_down", ks_dn))}
+    return out
+
+
 def run_prefill(args, dist, peaks, peak_src):
     import torch
     from bit_grouped_expert_router_b200 import synth
@@ -266,6 +299,7 @@ def run_prefill(args, dist, peaks, peak_src):
         a = (f_gu + f_dn) / t / 1e12
         gg = {"achieved_tflops": round(a, 1), "frac_of_peak": round(a / peak_tf, 4),
               "us_per_chunk": round(t * 1e6, 1)}
+        gg.update(tile_stats(layers, xs, shape, prof, clk))
     res = dict(value=value, ms=ms, clocks=clk, roofline=roof, kernels=prof, grouped_gemm=gg,
                launches=8 * chunks * n_layers * args.steps, shape=shape, n_layers=n_layers,
                tokens_per_step=tokens_per_step)

@@ -29,6 +29,8 @@ MOE_FLAG_DECODE_UNFUSED = 0x2
 MOE_FLAG_POISON_WORKSPACE = 0x4
 MOE_FLAG_HOST_SYNC_ROUTING = 0x8
 MOE_FLAG_DEQUANT_TO_HBM = 0x10
+MOE_FLAG_NO_ROUTER = 0x20
+MOE_FLAG_NO_EXPERTS = 0x40
 MOE_FLAG_TEST_STALL = 0x100
 
 _ERR_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DEVICE", 3: "TOO_LARGE", 4: "CUDA",
@@ -85,8 +87,11 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_enable.argtypes = [P, ctypes.c_int]
         L.moe_profile_read.argtypes = [P, P, P]
         L.moe_route_static.argtypes = [P, I32, I32, P, P, I32, I32, P, P, P]
+        L.moe_forward_routed.argtypes = [P, P, I32, P, P, P, P, P]
+        L.moe_combine_rows.argtypes = [P, P, I32, P, I32, I32, P, P, P]
         for n in ("moe_create", "moe_forward", "moe_forward_host", "moe_forward_host_async", "moe_route", "moe_status",
-                  "moe_debug_copy", "moe_profile_enable", "moe_profile_read", "moe_route_static"):
+                  "moe_debug_copy", "moe_profile_enable", "moe_profile_read", "moe_route_static",
+                  "moe_forward_routed", "moe_combine_rows"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -175,6 +180,27 @@ class Layer:
         check(lib().moe_forward_host_async(self.handle, _ptr(x_host), x_host.shape[0], _ptr(out_host),
                                            _stream_ptr(stream)))
         return out_host
+
+    def forward_routed(self, x, idx, gates, shared_gate=None, out=None, stream=None):
+        """out[T, H] bf16 = sum_j gates[:, j] FFN_{idx[:, j]}(x) (+ shared_gate FFN_shared(x)) with the
+        routing given: idx [T, k] int32, gates [T, k] fp32, shared_gate [T] fp32 (has_shared)."""
+        import torch
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x.device)
+        check(lib().moe_forward_routed(self.handle, _ptr(x), T, _ptr(idx), _ptr(gates), _ptr(shared_gate),
+                                       _ptr(out), _stream_ptr(stream)))
+        return out
+
+    def combine_rows(self, rows, pos, base=None, out=None, stream=None):
+        """out[T, H] bf16 = base + sum over j of rows[pos[:, j]] (pos < 0: no row), fp32 sums."""
+        import torch
+        T, k = pos.shape
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=pos.device)
+        check(lib().moe_combine_rows(self.handle, _ptr(rows), rows.shape[0], _ptr(pos), T, k, _ptr(base),
+                                     _ptr(out), _stream_ptr(stream)))
+        return out
 
     def route(self, x, stream=None):
         """-> dict(idx [T,k] int32, gates [T,k] f32, shared_gate [T] f32, offsets [E+1] int32,

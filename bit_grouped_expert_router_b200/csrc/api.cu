@@ -104,8 +104,9 @@ Layout make_layout(const moe_config& c) {
     L.max_tiles = (L.rows_cap + 127) / 128 + L.G;   // tiles of >= 128 rows (gemm_tile_rows)
     const size_t per_mat_gu = (size_t)(L.I / 64) * (L.H / 64) * kBlockBytes;   // gate+up rows 2I
     const size_t per_mat_dn = (size_t)(L.H / 128) * (L.I / 64) * kBlockBytes;
-    L.w_gu_bytes = per_mat_gu * L.G;
-    L.w_dn_bytes = per_mat_dn * L.G;
+    const bool experts = !(c.flags & MOE_FLAG_NO_EXPERTS);
+    L.w_gu_bytes = experts ? per_mat_gu * L.G : 0;
+    L.w_dn_bytes = experts ? per_mat_dn * L.G : 0;
     // router region: transposed fp32 [H][E], bias [E], shared-gate vector [H], public-layout fp32
     // copy [E][H]; every sub-buffer starts on a 256-byte boundary (vector loads need 16 B)
     L.o_wrt = 0;
@@ -174,8 +175,13 @@ int validate_config(const moe_config* c) {
     if ((c->decode_max_tokens >= 2 || (c->flags & MOE_FLAG_DECODE_UNFUSED)) && c->top_k + c->has_shared > 16)
         return fail(MOE_ERR_INVALID_ARG, "the multi-kernel decode path supports top_k + has_shared <= 16");
     if (c->flags & ~(uint32_t)(MOE_FLAG_ROUTER_SIMT | MOE_FLAG_DECODE_UNFUSED | MOE_FLAG_POISON_WORKSPACE |
-                               MOE_FLAG_HOST_SYNC_ROUTING | MOE_FLAG_DEQUANT_TO_HBM | MOE_FLAG_TEST_STALL))
+                               MOE_FLAG_HOST_SYNC_ROUTING | MOE_FLAG_DEQUANT_TO_HBM | MOE_FLAG_NO_ROUTER |
+                               MOE_FLAG_NO_EXPERTS | MOE_FLAG_TEST_STALL))
         return fail(MOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
+    if ((c->flags & MOE_FLAG_NO_ROUTER) && (c->flags & MOE_FLAG_NO_EXPERTS))
+        return fail(MOE_ERR_INVALID_ARG, "MOE_FLAG_NO_ROUTER and MOE_FLAG_NO_EXPERTS leave nothing to run");
+    if ((c->flags & MOE_FLAG_NO_EXPERTS) && (c->flags & MOE_FLAG_DEQUANT_TO_HBM))
+        return fail(MOE_ERR_INVALID_ARG, "MOE_FLAG_DEQUANT_TO_HBM needs expert weights");
     return MOE_OK;
 }
 
@@ -325,6 +331,43 @@ int enqueue_routing(moe_handle* h, Prof& pf, const Ctx& c, bool decode, cudaStre
     return MOE_OK;
 }
 
+// The expert steps of a call after routing: the GEMV chain (decode) or the gather, the two grouped
+// GEMMs and the finalisation (prefill).
+int enqueue_experts(moe_handle* h, Prof& pf, const Ctx& c, bool decode, cudaStream_t st) {
+    if (decode) {
+        MOE_LAUNCH("moe.gemv_gateup", launch_gemv_gateup(c, st));
+        pf.mark(7);
+        MOE_LAUNCH("moe.gemv_down", launch_gemv_down(c, st));
+        pf.mark(8);
+    } else {
+        MOE_LAUNCH("moe.gather_rows", launch_gather_rows(c, h->num_sms, st));
+        pf.mark(10);
+        int sms_gu = h->num_sms, sms_dn = h->num_sms;
+        if (h->cfg.flags & MOE_FLAG_HOST_SYNC_ROUTING) {
+            // ablation of GPU-resident routing: the host waits for the routing kernels, reads the
+            // tile count back and sizes the grouped GEMMs' grids from it (same results)
+            int nt = 0;
+            {
+                NvtxRange r("moe.host_sync_routing");
+                CUDA_TRY(cudaMemcpyAsync(&nt, c.ntiles, sizeof(int), cudaMemcpyDeviceToHost, st));
+                CUDA_TRY(cudaStreamSynchronize(st));
+            }
+            const int per_cta = c.tile_rows == 128 ? 2 : 1;   // CTAs per SM of the launch shape
+            auto sms_for = [&](int tasks) { return std::max(1, std::min(h->num_sms, (tasks + per_cta - 1) / per_cta)); };
+            sms_gu = sms_for(nt * (h->L.I / 64));
+            sms_dn = sms_for(nt * (h->L.H / 128));
+        }
+        const bool a16 = h->w16 != nullptr;
+        MOE_LAUNCH("moe.gemm_gateup", launch_gemm_gateup(c, h->maps_gu, a16 ? &h->amap_gu : nullptr, sms_gu, st));
+        pf.mark(4);
+        MOE_LAUNCH("moe.gemm_down", launch_gemm_down(c, h->maps_dn, a16 ? &h->amap_dn : nullptr, sms_dn, st));
+        pf.mark(5);
+        MOE_LAUNCH("moe.finalize", launch_finalize(c, st));
+        pf.mark(6);
+    }
+    return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -349,17 +392,24 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     int rc = validate_config(cfg);
     if (rc != MOE_OK) return rc;
     if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
-    const void* req[] = {w->q_gate, w->q_up, w->q_down, w->s_gate, w->b_gate, w->s_up, w->b_up, w->s_down, w->b_down,
-                         w->router};
-    for (const void* p : req)
-        if (!p || !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "a required weight pointer is NULL or misaligned");
-    if (cfg->has_shared) {
-        const void* sh[] = {w->qs_gate, w->qs_up, w->qs_down, w->ss_gate, w->bs_gate, w->ss_up, w->bs_up,
-                            w->ss_down, w->bs_down, w->shared_gate};
-        for (const void* p : sh)
-            if (!p || !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "a shared-expert pointer is NULL or misaligned");
+    const bool experts = !(cfg->flags & MOE_FLAG_NO_EXPERTS), router = !(cfg->flags & MOE_FLAG_NO_ROUTER);
+    if (experts) {
+        const void* req[] = {w->q_gate, w->q_up, w->q_down, w->s_gate, w->b_gate, w->s_up, w->b_up, w->s_down, w->b_down};
+        for (const void* p : req)
+            if (!p || !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "a required weight pointer is NULL or misaligned");
+        if (cfg->has_shared) {
+            const void* sh[] = {w->qs_gate, w->qs_up, w->qs_down, w->ss_gate, w->bs_gate, w->ss_up, w->bs_up,
+                                w->ss_down, w->bs_down};
+            for (const void* p : sh)
+                if (!p || !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "a shared-expert pointer is NULL or misaligned");
+        }
     }
-    if (w->router_bias && !aligned16(w->router_bias)) return fail(MOE_ERR_INVALID_ARG, "router_bias misaligned");
+    if (router) {
+        if (!w->router || !aligned16(w->router)) return fail(MOE_ERR_INVALID_ARG, "router is NULL or misaligned");
+        if (cfg->has_shared && (!w->shared_gate || !aligned16(w->shared_gate)))
+            return fail(MOE_ERR_INVALID_ARG, "shared_gate is NULL or misaligned");
+        if (w->router_bias && !aligned16(w->router_bias)) return fail(MOE_ERR_INVALID_ARG, "router_bias misaligned");
+    }
 
     int ndev = 0;
     CUDA_TRY(cudaGetDeviceCount(&ndev));
@@ -427,7 +477,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     a.qs[0] = w->qs_gate; a.ss[0] = w->ss_gate; a.bs[0] = w->bs_gate;
     a.qs[1] = w->qs_up;   a.ss[1] = w->ss_up;   a.bs[1] = w->bs_up;
     a.dst = w_gu;
-    e = launch_repack(a, L.G, L.I / 64, L.H / 64, st);
+    e = experts ? launch_repack(a, L.G, L.I / 64, L.H / 64, st) : cudaSuccess;
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "repack gate/up: %s", cudaGetErrorString(e)));
     RepackArgs d{};
     d.E = L.E;
@@ -440,15 +490,20 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     d.qs[0] = w->qs_down; d.ss[0] = w->ss_down; d.bs[0] = w->bs_down;
     d.qs[1] = w->qs_down; d.ss[1] = w->ss_down; d.bs[1] = w->bs_down;
     d.dst = w_dn;
-    e = launch_repack(d, L.G, L.H / 128, L.I / 64, st);
+    e = experts ? launch_repack(d, L.G, L.H / 128, L.I / 64, st) : cudaSuccess;
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "repack down: %s", cudaGetErrorString(e)));
-    e = launch_router_prep(w->router, w->router_bias, cfg->has_shared ? w->shared_gate : nullptr, L.H, L.E, wrt, rbias,
-                           sgw, st);
-    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router prep: %s", cudaGetErrorString(e)));
-    e = cudaMemcpyAsync(router32, w->router, sizeof(float) * (size_t)L.E * L.H, cudaMemcpyDeviceToDevice, st);
-    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router copy: %s", cudaGetErrorString(e)));
-    e = launch_router_split(w->router, L.H, L.E, L.Epad, wsplit, st);
-    if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router split: %s", cudaGetErrorString(e)));
+    if (router) {
+        e = launch_router_prep(w->router, w->router_bias, cfg->has_shared ? w->shared_gate : nullptr, L.H, L.E, wrt,
+                               rbias, sgw, st);
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router prep: %s", cudaGetErrorString(e)));
+        e = cudaMemcpyAsync(router32, w->router, sizeof(float) * (size_t)L.E * L.H, cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router copy: %s", cudaGetErrorString(e)));
+        e = launch_router_split(w->router, L.H, L.E, L.Epad, wsplit, st);
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router split: %s", cudaGetErrorString(e)));
+    } else {
+        e = cudaMemsetAsync(rregion, 0, align_up(L.router_bytes, 256) + L.wsplit_bytes, st);
+        if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "router region: %s", cudaGetErrorString(e)));
+    }
     uint32_t flags_host[2] = {0, 0};
     e = cudaMemcpyAsync(flags_host, status, sizeof flags_host, cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -491,7 +546,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.dfz.cnt = reinterpret_cast<unsigned*>(ws + L.o_dfz_cnt);
     c.dfz.dirty = reinterpret_cast<unsigned*>(ws + L.o_dfz_dirty);
 
-    if (decode_fused_geometry(L.H, L.I, L.E, L.k, cfg->has_shared, &h->dgeom)) {
+    if (experts && router && decode_fused_geometry(L.H, L.I, L.E, L.k, cfg->has_shared, &h->dgeom)) {
         int nclusters = 0;
         e = decode_fused_prepare(h->dgeom);
         if (e == cudaSuccess) e = decode_fused_max_clusters(h->dgeom, &nclusters);
@@ -529,7 +584,10 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
 
 int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void* stream) {
     int rc = check_call(h, x, T, out, true);
-    if (rc != MOE_OK || T == 0) return rc;
+    if (rc != MOE_OK) return rc;
+    if (h->cfg.flags & (MOE_FLAG_NO_ROUTER | MOE_FLAG_NO_EXPERTS))
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward needs a handle with router and experts (see MOE_FLAG_NO_*)");
+    if (T == 0) return rc;
     NvtxRange range("moe_forward");
     DeviceGuard guard(h->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -552,44 +610,15 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     }
     rc = enqueue_routing(h, pf, c, decode, st);
     if (rc != MOE_OK) return rc;
-    if (decode) {
-        MOE_LAUNCH("moe.gemv_gateup", launch_gemv_gateup(c, st));
-        pf.mark(7);
-        MOE_LAUNCH("moe.gemv_down", launch_gemv_down(c, st));
-        pf.mark(8);
-    } else {
-        MOE_LAUNCH("moe.gather_rows", launch_gather_rows(c, h->num_sms, st));
-        pf.mark(10);
-        int sms_gu = h->num_sms, sms_dn = h->num_sms;
-        if (h->cfg.flags & MOE_FLAG_HOST_SYNC_ROUTING) {
-            // ablation of GPU-resident routing: the host waits for the routing kernels, reads the
-            // tile count back and sizes the grouped GEMMs' grids from it (same results)
-            int nt = 0;
-            {
-                NvtxRange r("moe.host_sync_routing");
-                CUDA_TRY(cudaMemcpyAsync(&nt, c.ntiles, sizeof(int), cudaMemcpyDeviceToHost, st));
-                CUDA_TRY(cudaStreamSynchronize(st));
-            }
-            const int per_cta = c.tile_rows == 128 ? 2 : 1;   // CTAs per SM of the launch shape
-            auto sms_for = [&](int tasks) { return std::max(1, std::min(h->num_sms, (tasks + per_cta - 1) / per_cta)); };
-            sms_gu = sms_for(nt * (h->L.I / 64));
-            sms_dn = sms_for(nt * (h->L.H / 128));
-        }
-        const bool a16 = h->w16 != nullptr;
-        MOE_LAUNCH("moe.gemm_gateup", launch_gemm_gateup(c, h->maps_gu, a16 ? &h->amap_gu : nullptr, sms_gu, st));
-        pf.mark(4);
-        MOE_LAUNCH("moe.gemm_down", launch_gemm_down(c, h->maps_dn, a16 ? &h->amap_dn : nullptr, sms_dn, st));
-        pf.mark(5);
-        MOE_LAUNCH("moe.finalize", launch_finalize(c, st));
-        pf.mark(6);
-    }
-    return MOE_OK;
+    return enqueue_experts(h, pf, c, decode, st);
 }
 
 int moe_forward_host_async(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t* out_host, void* stream) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
     if (T > h->cfg.max_tokens) return fail(MOE_ERR_TOO_LARGE, "T = %d exceeds max_tokens = %d", T, h->cfg.max_tokens);
+    if (h->cfg.flags & (MOE_FLAG_NO_ROUTER | MOE_FLAG_NO_EXPERTS))
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward needs a handle with router and experts (see MOE_FLAG_NO_*)");
     if (T == 0) return MOE_OK;
     if (!x_host || !out_host) return fail(MOE_ERR_INVALID_ARG, "host buffers must not be NULL");
     DeviceGuard guard(h->device);
@@ -604,6 +633,53 @@ int moe_forward_host_async(moe_handle* h, const uint16_t* x_host, int32_t T, uin
     return MOE_OK;
 }
 
+int moe_forward_routed(moe_handle* h, const uint16_t* x, int32_t T, const int32_t* idx, const float* gates,
+                       const float* shared_gate, uint16_t* out, void* stream) {
+    int rc = check_call(h, x, T, out, true);
+    if (rc != MOE_OK) return rc;
+    if (h->cfg.flags & MOE_FLAG_NO_EXPERTS)
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward_routed: handle created without expert weights");
+    if (T == 0) return MOE_OK;
+    if (!idx || !gates || !aligned16(idx) || !aligned16(gates))
+        return fail(MOE_ERR_INVALID_ARG, "idx and gates must be 16-byte aligned device pointers");
+    if (h->cfg.has_shared && (!shared_gate || !aligned16(shared_gate)))
+        return fail(MOE_ERR_INVALID_ARG, "shared_gate must be a 16-byte aligned device pointer (has_shared = 1)");
+    NvtxRange range("moe_forward_routed");
+    DeviceGuard guard(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    const bool decode = use_decode(h, T);
+    const Ctx c = make_ctx(h, T, x, out, decode);
+    Prof pf(h, st);
+    MOE_LAUNCH("moe.routing_supplied", launch_routing_supplied(c, idx, gates, shared_gate, !decode, st));
+    pf.mark(1);
+    if (!decode) {
+        MOE_LAUNCH("moe.bucket_scan", launch_bucket_scan(c, st));
+        pf.mark(2);
+        MOE_LAUNCH("moe.scatter", launch_scatter(c, st));
+        pf.mark(3);
+    }
+    return enqueue_experts(h, pf, c, decode, st);
+}
+
+int moe_combine_rows(moe_handle* h, const uint16_t* rows, int32_t n_rows, const int32_t* pos, int32_t T, int32_t k,
+                     const uint16_t* base, uint16_t* out, void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "T and n_rows must be >= 0");
+    if (k < 1 || k > 32) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, 32]");
+    if (T == 0) return MOE_OK;
+    if (!pos || !aligned16(pos) || !out || !aligned16(out) || (base && !aligned16(base)) ||
+        (n_rows > 0 && (!rows || !aligned16(rows))))
+        return fail(MOE_ERR_INVALID_ARG, "pointers must be 16-byte aligned device pointers");
+    NvtxRange range("moe_combine_rows");
+    DeviceGuard guard(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    MOE_LAUNCH("moe.combine_rows", launch_combine_rows(rows, n_rows, pos, T, k, h->L.H, base, out, h->base.status,
+                                                       h->num_sms, st));
+    return MOE_OK;
+}
+
 int moe_forward_host(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t* out_host, void* stream) {
     const int rc = moe_forward_host_async(h, x_host, T, out_host, stream);
     if (rc != MOE_OK || T == 0) return rc;
@@ -615,7 +691,9 @@ int moe_forward_host(moe_handle* h, const uint16_t* x_host, int32_t T, uint16_t*
 int moe_route(moe_handle* h, const uint16_t* x, int32_t T, int32_t* idx, float* gates, float* shared_gate,
               int32_t* offsets, int32_t* perm, void* stream) {
     int rc = check_call(h, x, T, nullptr, false);
-    if (rc != MOE_OK || T == 0) return rc;
+    if (rc != MOE_OK) return rc;
+    if (h->cfg.flags & MOE_FLAG_NO_ROUTER) return fail(MOE_ERR_INVALID_ARG, "moe_route: handle created without a router");
+    if (T == 0) return rc;
     DeviceGuard guard(h->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;

@@ -49,6 +49,8 @@
 // TMEM: two fp32 accumulators of kBN columns.  Every wait is bounded (common.cuh); on a timeout the
 // roles unwind, the producer waits for its copies in flight, the MMA thread waits for its MMAs,
 // and warp 1 frees the TMEM.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -551,6 +553,62 @@ __global__ void __launch_bounds__(256) finalize_kernel(Ctx c) {
         o.w = *reinterpret_cast<uint32_t*>(&p3);
         reinterpret_cast<uint4*>(c.out)[i] = o;
     }
+}
+
+// out[t] = bf16(base[t] + sum over j of rows[pos[t][j]]), fp32 sums in j order, 8 elements per
+// thread per step; pos < 0 is no row, pos >= n_rows is recorded (BOUNDS) and skipped.
+__global__ void __launch_bounds__(256) combine_rows_kernel(const uint16_t* __restrict__ rows, int n_rows,
+                                                           const int* __restrict__ pos, int T, int k, int H,
+                                                           const uint16_t* __restrict__ base, uint16_t* __restrict__ out,
+                                                           uint32_t* status) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int n8 = H / 8;
+    const size_t total = (size_t)T * n8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t t = i / n8;
+        const int ch = (int)(i % n8);
+        float a[8];
+        uint4 b = make_uint4(0u, 0u, 0u, 0u);
+        if (base) b = *reinterpret_cast<const uint4*>(base + t * H + ch * 8);
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            a[2 * u] = __uint_as_float(bw[u] << 16);
+            a[2 * u + 1] = __uint_as_float(bw[u] & 0xFFFF0000u);
+        }
+        for (int j = 0; j < k; ++j) {
+            const int p = pos[t * k + j];
+            if (p < 0) continue;
+            if (p >= n_rows) {
+                set_status(status, MOE_STATUS_BOUNDS);
+                continue;
+            }
+            const uint4 r = *reinterpret_cast<const uint4*>(rows + (size_t)p * H + ch * 8);
+            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                a[2 * u] += __uint_as_float(rw[u] << 16);
+                a[2 * u + 1] += __uint_as_float(rw[u] & 0xFFFF0000u);
+            }
+        }
+        uint32_t ow[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            __nv_bfloat162 v = __floats2bfloat162_rn(a[2 * u], a[2 * u + 1]);
+            ow[u] = *reinterpret_cast<uint32_t*>(&v);
+        }
+        *reinterpret_cast<uint4*>(out + t * H + ch * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
+cudaError_t launch_combine_rows(const uint16_t* rows, int n_rows, const int* pos, int T, int k, int H,
+                                const uint16_t* base, uint16_t* out, uint32_t* status, int num_sms, cudaStream_t st) {
+    const size_t total = (size_t)T * (H / 8);
+    const size_t want = (total + 255) / 256;
+    const int blocks = (int)std::min<size_t>(want > 0 ? want : 1, (size_t)num_sms * 16);
+    return launch_pdl(combine_rows_kernel, dim3(blocks), dim3(256), 0, st, rows, n_rows, pos, T, k, H, base, out,
+                      status);
 }
 
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st) {

@@ -108,6 +108,8 @@ cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmW, const CUtenso
 int router_tc_smem_bytes();
 int router_tc_splits();
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
+cudaError_t launch_routing_supplied(const Ctx& c, const int* idx, const float* gates, const float* sg,
+                                    bool prefill, cudaStream_t st);
 cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st);
 
@@ -137,6 +139,8 @@ cudaError_t launch_gemm_down(const Ctx& c, const TokenMaps& maps, const CUtensor
 cudaError_t launch_dequant_rows(const uint8_t* blocks, int groups, int m_tiles, int k_steps, __half* dst,
                                 cudaStream_t st);
 cudaError_t launch_finalize(const Ctx& c, cudaStream_t st);
+cudaError_t launch_combine_rows(const uint16_t* rows, int n_rows, const int* pos, int T, int k, int H,
+                                const uint16_t* base, uint16_t* out, uint32_t* status, int num_sms, cudaStream_t st);
 // Token rows per grouped-GEMM tile for a call of T tokens: 128 (two CTAs per SM) when the
 // routed experts average at most 64 tokens (T * k <= 64 * E), else 256 (one CTA per SM).
 int gemm_tile_rows(int T, int k, int E);

@@ -102,6 +102,64 @@ __device__ __forceinline__ uint32_t ord_key(float v) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The per-token row pass of the routing step, one warp per token: optionally the shared-expert
+// gate sigmoid(x_t . shared_gate) (dot), and on the prefill path the fp16 copy of the row for the
+// tensor cores (range-checked) and the zeroing of the token's fp32 combine row.  Returns the gate
+// (0 without dot) in every lane.
+__device__ float token_row_pass(const Ctx& c, int t, int lane, bool dot, bool prefill) {
+    float sgv = 0.f;
+    const uint16_t* xr = c.x + (size_t)t * c.H;
+    float d = 0.f;
+    bool range_bad = false;
+    if (dot || prefill) {
+        // the lane's row loads (up to 8 chunks of 8 elements) are all issued before the arithmetic
+        constexpr int kXU = 8;
+        for (int h0 = lane * 8; h0 < c.H; h0 += 256 * kXU) {
+            uint4 rawv[kXU];
+#pragma unroll
+            for (int u = 0; u < kXU; ++u)
+                if (h0 + 256 * u < c.H) rawv[u] = __ldg(reinterpret_cast<const uint4*>(xr + h0 + 256 * u));
+#pragma unroll
+            for (int u = 0; u < kXU; ++u) {
+                const int h = h0 + 256 * u;
+                if (h >= c.H) break;
+                const uint4 raw = rawv[u];
+                if (dot) {
+                    const float4 w0 = *reinterpret_cast<const float4*>(c.sgw + h);
+                    const float4 w1 = *reinterpret_cast<const float4*>(c.sgw + h + 4);
+                    d = fmaf(__uint_as_float(raw.x << 16), w0.x, d);
+                    d = fmaf(__uint_as_float(raw.x & 0xFFFF0000u), w0.y, d);
+                    d = fmaf(__uint_as_float(raw.y << 16), w0.z, d);
+                    d = fmaf(__uint_as_float(raw.y & 0xFFFF0000u), w0.w, d);
+                    d = fmaf(__uint_as_float(raw.z << 16), w1.x, d);
+                    d = fmaf(__uint_as_float(raw.z & 0xFFFF0000u), w1.y, d);
+                    d = fmaf(__uint_as_float(raw.w << 16), w1.z, d);
+                    d = fmaf(__uint_as_float(raw.w & 0xFFFF0000u), w1.w, d);
+                }
+                if (prefill) {   // fp16 copy of the row for the tensor-core path (exact for |x| < 65504)
+                    uint4 o;
+                    o.x = bf16x2_to_half2_bits(raw.x, &range_bad);
+                    o.y = bf16x2_to_half2_bits(raw.y, &range_bad);
+                    o.z = bf16x2_to_half2_bits(raw.z, &range_bad);
+                    o.w = bf16x2_to_half2_bits(raw.w, &range_bad);
+                    *reinterpret_cast<uint4*>(c.x16 + (size_t)t * c.H + h) = o;
+                }
+            }
+        }
+    }
+    if (dot) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        sgv = 1.f / (1.f + expf(-d));
+    }
+    if (range_bad) set_status(c.status, MOE_STATUS_RANGE);
+    if (prefill) {
+        float4* ar = reinterpret_cast<float4*>(c.acc + (size_t)t * c.H);
+        for (int h4 = lane; h4 < c.H / 4; h4 += 32) ar[h4] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return sgv;
+}
+
 __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
     griddep_wait();
     griddep_launch_dependents();
@@ -182,61 +240,47 @@ __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
         c.gates[(size_t)t * c.k + lane] = p / z;
         if (do_hist) atomicAdd(&c.hist[(size_t)(t / kTokPerBucketBlk) * c.E + my_e], 1);
     }
-    float sgv = 0.f;
-    const uint16_t* xr = c.x + (size_t)t * c.H;
-    float d = 0.f;
-    bool range_bad = false;
-    if (c.has_shared || do_hist) {
-        // the lane's row loads (up to 8 chunks of 8 elements) are all issued before the arithmetic
-        constexpr int kXU = 8;
-        for (int h0 = lane * 8; h0 < c.H; h0 += 256 * kXU) {
-            uint4 rawv[kXU];
-#pragma unroll
-            for (int u = 0; u < kXU; ++u)
-                if (h0 + 256 * u < c.H) rawv[u] = __ldg(reinterpret_cast<const uint4*>(xr + h0 + 256 * u));
-#pragma unroll
-            for (int u = 0; u < kXU; ++u) {
-                const int h = h0 + 256 * u;
-                if (h >= c.H) break;
-                const uint4 raw = rawv[u];
-                if (c.has_shared) {
-                    const float4 w0 = *reinterpret_cast<const float4*>(c.sgw + h);
-                    const float4 w1 = *reinterpret_cast<const float4*>(c.sgw + h + 4);
-                    d = fmaf(__uint_as_float(raw.x << 16), w0.x, d);
-                    d = fmaf(__uint_as_float(raw.x & 0xFFFF0000u), w0.y, d);
-                    d = fmaf(__uint_as_float(raw.y << 16), w0.z, d);
-                    d = fmaf(__uint_as_float(raw.y & 0xFFFF0000u), w0.w, d);
-                    d = fmaf(__uint_as_float(raw.z << 16), w1.x, d);
-                    d = fmaf(__uint_as_float(raw.z & 0xFFFF0000u), w1.y, d);
-                    d = fmaf(__uint_as_float(raw.w << 16), w1.z, d);
-                    d = fmaf(__uint_as_float(raw.w & 0xFFFF0000u), w1.w, d);
-                }
-                if (do_hist) {   // fp16 copy of the row for the tensor-core path (exact for |x| < 65504)
-                    uint4 o;
-                    o.x = bf16x2_to_half2_bits(raw.x, &range_bad);
-                    o.y = bf16x2_to_half2_bits(raw.y, &range_bad);
-                    o.z = bf16x2_to_half2_bits(raw.z, &range_bad);
-                    o.w = bf16x2_to_half2_bits(raw.w, &range_bad);
-                    *reinterpret_cast<uint4*>(c.x16 + (size_t)t * c.H + h) = o;
-                }
-            }
-        }
-    }
-    if (c.has_shared) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        sgv = 1.f / (1.f + expf(-d));
-    }
-    if (range_bad) set_status(c.status, MOE_STATUS_RANGE);
+    const float sgv = token_row_pass(c, t, lane, c.has_shared != 0, do_hist != 0);
     if (lane == 0) c.sg[t] = sgv;
-    if (do_hist) {
-        float4* ar = reinterpret_cast<float4*>(c.acc + (size_t)t * c.H);
-        for (int h4 = lane; h4 < c.H / 4; h4 += 32) ar[h4] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 }
 
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st) {
     return launch_pdl(topk_kernel, dim3((c.T + 7) / 8), dim3(256), 0, st, c, histogram ? 1 : 0);
+}
+
+// Routing supplied by the caller (moe_forward_routed): the same outputs as topk_kernel -- expert
+// ids, gates and shared gate in the workspace, the bucketing histogram and the row pass on the
+// prefill path -- with idx / gates / shared gate read instead of selected.  An id outside [0, E)
+// is recorded (BOUNDS) and becomes expert 0 with gate 0, so it contributes nothing.
+__global__ void __launch_bounds__(256) routing_supplied_kernel(Ctx c, const int* __restrict__ idx_in,
+                                                               const float* __restrict__ gates_in,
+                                                               const float* __restrict__ sg_in, int prefill) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int lane = lane_id();
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= c.T) return;
+    if (lane < c.k) {
+        const size_t j = (size_t)t * c.k + lane;
+        int e = idx_in[j];
+        float g = gates_in[j];
+        if (e < 0 || e >= c.E) {
+            set_status(c.status, MOE_STATUS_BOUNDS);
+            e = 0;
+            g = 0.f;
+        }
+        c.idx[j] = e;
+        c.gates[j] = g;
+        if (prefill) atomicAdd(&c.hist[(size_t)(t / kTokPerBucketBlk) * c.E + e], 1);
+    }
+    token_row_pass(c, t, lane, false, prefill != 0);
+    if (lane == 0) c.sg[t] = c.has_shared ? sg_in[t] : 0.f;
+}
+
+cudaError_t launch_routing_supplied(const Ctx& c, const int* idx, const float* gates, const float* sg, bool prefill,
+                                    cudaStream_t st) {
+    return launch_pdl(routing_supplied_kernel, dim3((c.T + 7) / 8), dim3(256), 0, st, c, idx, gates, sg,
+                      prefill ? 1 : 0);
 }
 
 // ---- bucket scan + tile list (one CTA) ---------------------------------------------------------

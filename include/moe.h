@@ -90,6 +90,15 @@ extern "C" {
                                           the handle's memory (4x the bytes of the packed codes),
                                           and the prefill grouped GEMMs load those instead of
                                           rebuilding each tile from the 4-bit blocks (same results) */
+#define MOE_FLAG_NO_ROUTER       0x20u /* a handle without a router: router, router_bias and
+                                          shared_gate may be NULL and are not read; the handle
+                                          serves moe_forward_routed (and moe_combine_rows) only,
+                                          e.g. one rank's shard of experts in expert parallelism */
+#define MOE_FLAG_NO_EXPERTS      0x40u /* a handle without expert weights: the q_*, s_*, b_* and
+                                          shared-expert pointers may be NULL and are not read, no
+                                          memory is allocated for them, and the handle serves
+                                          moe_route (and moe_combine_rows) only: the router of an
+                                          expert-parallel layer whose experts live on other GPUs */
 #define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its loads on
                                           every call, and the fused batch-1 decode kernel withholds
                                           one router result on the handle's first call, so bounded
@@ -188,6 +197,32 @@ MOE_API int moe_forward_host_async(moe_handle *h, const uint16_t *x_host, int32_
  * Errors as for moe_forward. */
 MOE_API int moe_route(moe_handle *h, const uint16_t *x, int32_t T, int32_t *idx, float *gates,
               float *shared_gate, int32_t *offsets, int32_t *perm, void *stream);
+
+/* Source: the forward pass defined at the top of this file with its routing step supplied by the
+ * caller; the expert-parallel form of the layer (experts sharded over GPUs, rows dispatched to
+ * the GPU that holds their expert) calls it on each shard (library design; the pages run one GPU).
+ * out[T, H] (bf16) = for each row t of x[T, H] (bf16):
+ *     sum_j gates[t, j] FFN_{idx[t, j]}(x_t)  +  shared_gate[t] FFN_shared(x_t)   (bf16 rounding)
+ * with idx[T, k] int32 in [0, E) and gates[T, k] fp32 given by the caller (any values: no top-k,
+ * no renormalisation, an expert may repeat within a row) and shared_gate[T] fp32 (NULL when
+ * has_shared == 0; required otherwise).  The same kernels as moe_forward run after the routing
+ * step (grouped GEMMs for T > decode_max_tokens, the GEMV chain otherwise).  An idx entry outside
+ * [0, E) contributes nothing and is reported as MOE_ERR_DEVICE_BOUNDS by moe_status.
+ * Errors: INVALID_ARG (null/misaligned pointer, handle created with MOE_FLAG_NO_EXPERTS),
+ * TOO_LARGE, CUDA. */
+MOE_API int moe_forward_routed(moe_handle *h, const uint16_t *x, int32_t T, const int32_t *idx,
+                               const float *gates, const float *shared_gate, uint16_t *out, void *stream);
+
+/* Source: the combine step of the forward pass (out_t = sum of the gated expert outputs) for rows
+ * that come back from other GPUs in expert parallelism (library design).
+ * out[T, H] (bf16) = bf16( base[t] + sum over j < k with pos[t, j] >= 0 of rows[pos[t, j]] ),
+ * summed in fp32 in j order, for rows[n_rows, H] bf16, pos[T, k] int32 and base[T, H] bf16 (or
+ * NULL for zeros), all device pointers; out may not alias rows or base.  Uses the handle's device
+ * and status word only (any handle with matching H).  A pos entry >= n_rows is skipped and
+ * reported as MOE_ERR_DEVICE_BOUNDS by moe_status.
+ * Errors: INVALID_ARG (null/misaligned pointer, k outside [1, 32], n_rows < 0), CUDA. */
+MOE_API int moe_combine_rows(moe_handle *h, const uint16_t *rows, int32_t n_rows, const int32_t *pos,
+                             int32_t T, int32_t k, const uint16_t *base, uint16_t *out, void *stream);
 
 /* Source: library convenience (no passage).
  * Synchronise the stream of the handle's last call, read and clear the device status word.

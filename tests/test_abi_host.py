@@ -45,7 +45,8 @@ def test_device_bytes_counts_the_repacked_layer(lib):
 
 @pytest.mark.parametrize("bad", [dict(group=32), dict(H=200), dict(I=96), dict(E=0), dict(E=300),
                                  dict(k=0), dict(k=33, E=64), dict(k=9, E=8), dict(max_tokens=0),
-                                 dict(decode_max_tokens=-1), dict(decode_max_tokens=65536), dict(flags=0x40), dict(flags=0x200),
+                                 dict(decode_max_tokens=-1), dict(decode_max_tokens=65536), dict(flags=0x80), dict(flags=0x200),
+                                 dict(flags=0x60), dict(flags=0x50),
                                  dict(k=16, decode_max_tokens=2)])
 def test_invalid_config_is_rejected_before_any_cuda_call(lib, bad):
     cfg = _cfg(**bad)
@@ -72,7 +73,30 @@ def test_null_handle_calls(lib):
     assert lib.moe_forward_host(None, None, 1, None, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_forward_host_async(None, None, 1, None, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_copy(None, 0, None, 0, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_routed(None, None, 1, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_rows(None, None, 0, None, 1, 1, None, None, None) == M.MOE_ERR_INVALID_ARG
     lib.moe_destroy(None)
+
+
+def test_router_only_handle_owns_no_expert_weights(lib):
+    full = lib.moe_device_bytes(ctypes.byref(_cfg()))
+    router_only = lib.moe_device_bytes(ctypes.byref(_cfg(flags=M.MOE_FLAG_NO_EXPERTS)))
+    per_expert = 1769472 * 257   # packed codes + fp16 scale/bias pairs of 256 experts + the shared one
+    assert full - router_only >= per_expert
+    assert lib.moe_device_bytes(ctypes.byref(_cfg(flags=M.MOE_FLAG_NO_ROUTER))) == full
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_router_only_create_needs_only_router_pointers(lib):
+    # only the router pointers are checked before the device: NULL expert weights pass validation
+    fake = ctypes.c_void_p(0x1000).value
+    w = M.MoeWeights(router=fake, shared_gate=fake)
+    h = ctypes.c_void_p()
+    rc = lib.moe_create(ctypes.byref(_cfg(flags=M.MOE_FLAG_NO_EXPERTS)), ctypes.byref(w), 0, None, ctypes.byref(h))
+    assert rc == M.MOE_ERR_CUDA, lib.moe_last_error().decode()
+    w2 = M.MoeWeights(q_gate=fake)
+    rc = lib.moe_create(ctypes.byref(_cfg(flags=M.MOE_FLAG_NO_EXPERTS)), ctypes.byref(w2), 0, None, ctypes.byref(h))
+    assert rc == M.MOE_ERR_INVALID_ARG and "router" in lib.moe_last_error().decode()
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
