@@ -13,7 +13,7 @@ from bit_grouped_expert_router_b200 import build as B
 from bit_grouped_expert_router_b200 import synth
 from bit_grouped_expert_router_b200.ep import Exchange, ExpertParallelLayer, LibraryShard
 from helpers import gapped_x
-from parity import compare
+from parity import compare, ulp_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +54,10 @@ def test_routed_forward_with_the_layers_own_routing_equals_forward(shape, T):
     want = layer.forward(xd)
     torch.cuda.synchronize()
     assert layer.status() == M.MOE_OK
-    assert torch.equal(got, want)
+    # the same kernels after the routing step; the combine's fp32 atomic sums may land in another
+    # order, so the two agree to one bf16 rounding step, and both match the oracle
+    g64, w64 = got.cpu().double().numpy(), want.cpu().double().numpy()
+    assert (np.abs(g64 - w64) <= ulp_bf16(np.maximum(np.abs(g64), np.abs(w64)))).all()
     compare(got.cpu(), ol.forward(x))
     layer.close()
 
@@ -191,8 +194,9 @@ def test_expert_parallel_one_rank_matches_the_oracle_and_forward(shape):
     layer = M.Layer.from_shape(_cuda(w), shape, max_tokens=512)
     ref = layer.forward(x.cuda()).cpu()
     layer.close()
-    # the same experts per row, summed as bf16 terms instead of in fp32: close, not identical
-    assert (out.cpu().float() - ref.float()).abs().max() < 2e-2
+    # the same experts per row, each gated term rounded to bf16 before the fp32 sum instead of
+    # summed in fp32 first: within the output tolerance of the single-GPU forward too
+    compare(out.cpu(), ref.double().numpy())
 
 
 @pytest.mark.parametrize("world", [2, 4])
