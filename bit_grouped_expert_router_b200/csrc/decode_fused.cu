@@ -280,6 +280,25 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                      kBlockBytes, bar_d);
         }
     };
+    // the routed unit's whole wave from the warp that picked the expert, one copy per lane (a
+    // bulk copy costs its issuing thread ~290 cycles, so one lane per copy issues them at once):
+    // lanes 0 .. nch-1 a gate/up chunk each, lanes 16 .. 16 + DM - 1 a down block each
+    auto issue_wave = [&](int e) {   // called by a whole warp
+        if (lane < g.nch) {
+            const uint8_t* gu = c.w_gu + ((size_t)(e * g.MTg + mt) * KSg + (size_t)g.KH * r) * kBlockBytes;
+            const int b0 = lane * g.KH / g.nch, b1 = (lane + 1) * g.KH / g.nch;
+            mbar_arrive_expect_tx(&bar_g[lane], (uint32_t)((b1 - b0) * kBlockBytes));
+            bulk_g2s(s.wgu + (size_t)b0 * kBlockBytes, gu + (size_t)b0 * kBlockBytes, (uint32_t)((b1 - b0) * kBlockBytes),
+                     &bar_g[lane]);
+        }
+        if (lane == 16) mbar_arrive_expect_tx(bar_d, (uint32_t)(g.DM * kBlockBytes));
+        __syncwarp();
+        if (lane >= 16 && lane - 16 < g.DM) {
+            const int b = lane - 16, mtd = g.DM * (int)r + b;
+            bulk_g2s(s.wdn + (size_t)b * kBlockBytes, c.w_dn + ((size_t)(e * MTd + mtd) * KSd + mt) * kBlockBytes,
+                     kBlockBytes, bar_d);
+        }
+    };
     const bool need_r = nrows > 0 || need_sg;
     if (need_r && warp == 2 && lane == 0) {
         mbar_arrive_expect_tx(bar_r, (uint32_t)((nrows + (need_sg ? 1 : 0)) * H * sizeof(float)));
@@ -316,19 +335,6 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     __syncthreads();
     const uint32_t tag = (uint32_t)s.ints[kIntTag];
     const bool dirty = s.ints[kIntDirty] != 0;
-    // per-group scaling of the input-column half this CTA's gate/up blocks cover
-    for (int grp = g.KH * (int)r + warp; grp < g.KH * ((int)r + 1); grp += kDWarps) {
-        const float a0 = s.xraw[64 * grp + 2 * lane], a1 = s.xraw[64 * grp + 2 * lane + 1];
-        const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(a0), fabsf(a1)))));
-        const float hs = half_warp_sum(a0 + a1);
-        const int K = 125 - group_exponent(m);
-        const float f1 = pow2f(K / 2), f2 = pow2f(K - K / 2);
-        const int e0 = 2 * lane, e1 = 2 * lane + 1;
-        s.xs[64 * grp + (e0 & ~7) + slot_of(e0 & 7)] = a0 * f1 * f2;
-        s.xs[64 * grp + (e1 & ~7) + slot_of(e1 & 7)] = a1 * f1 * f2;
-        if ((lane & 15) == 0) s.xsum[2 * grp + (lane >> 4)] = hs;
-        if (lane == 0) s.xsc[grp] = pow2f(149 - K);
-    }
     // a call after one that gave up part-way: the routed CTAs put the accumulator and the chunk
     // counters back to zero (ordered before their router words by a fence)
     if (dirty && routed) {
@@ -373,20 +379,45 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
             atomicOr(c.dfz.dirty, 1u);
         }
     }
-    if (routed && ok && tid < nrows) {
-        const int e = cr + g.NR * tid;
+    if (routed && ok && warp == 0) {
+        // the per-warp partial dots of each router row, summed across warp 0's lanes
+        float zr[kMaxRouterRows];
+#pragma unroll
+        for (int i = 0; i < kMaxRouterRows; ++i) {
+            zr[i] = (lane < kDWarps && i < nrows) ? s.red[kDWarps + lane * kMaxRouterRows + i] : 0.f;
+            zr[i] = warp_sum(zr[i]);
+        }
         float z = 0.f;
-        for (int w = 0; w < kDWarps; ++w) z += s.red[kDWarps + w * kMaxRouterRows + tid];
+#pragma unroll
+        for (int i = 0; i < kMaxRouterRows; ++i)
+            if (lane == i) z = zr[i];
         z += my_bias;
-        const bool stall = (c.flags & 0x100u) && cr == 0 && tag == 1u;   // test only: first call withholds
-        // the word carries its own data; after a failed call it must also follow this CTA's zeroing
-        if (dirty) fence_acq_rel_gpu();
-        if (!stall) st_relaxed_u64(c.dfz.slots + e, ((unsigned long long)tag << 32) | __float_as_uint(z));
+        if (lane < nrows) {
+            const int e = cr + g.NR * lane;
+            const bool stall = (c.flags & 0x100u) && cr == 0 && tag == 1u;   // test only: first call withholds
+            // the word carries its own data; after a failed call it must also follow this CTA's zeroing
+            if (dirty) fence_acq_rel_gpu();
+            if (!stall) st_relaxed_u64(c.dfz.slots + e, ((unsigned long long)tag << 32) | __float_as_uint(z));
+        }
     }
     if (need_sg && tid == 32) {
         float zz = 0.f;
         for (int w = 0; w < kDWarps; ++w) zz += s.red[w];
         s.misc[kMiscSgDot] = 1.f / (1.f + expf(-zz));
+    }
+    // per-group scaling of the input-column half this CTA's gate/up blocks cover (only the gate/up
+    // GEMV reads it, so it follows the router publish)
+    for (int grp = g.KH * (int)r + warp; grp < g.KH * ((int)r + 1); grp += kDWarps) {
+        const float a0 = s.xraw[64 * grp + 2 * lane], a1 = s.xraw[64 * grp + 2 * lane + 1];
+        const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(a0), fabsf(a1)))));
+        const float hs = half_warp_sum(a0 + a1);
+        const int K = 125 - group_exponent(m);
+        const float f1 = pow2f(K / 2), f2 = pow2f(K - K / 2);
+        const int e0 = 2 * lane, e1 = 2 * lane + 1;
+        s.xs[64 * grp + (e0 & ~7) + slot_of(e0 & 7)] = a0 * f1 * f2;
+        s.xs[64 * grp + (e1 & ~7) + slot_of(e1 & 7)] = a1 * f1 * f2;
+        if ((lane & 15) == 0) s.xsum[2 * grp + (lane >> 4)] = hs;
+        if (lane == 0) s.xsc[grp] = pow2f(149 - K);
     }
     if (ok && (routed || dirty) && warp == 0) {
         // every router word of this call: relaxed polls (each word carries its data; no load is
@@ -465,8 +496,8 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
             if (lane == 0) {
                 s.ints[kIntSel] = sel;
                 s.misc[kMiscGate] = gsel;
-                issue_gateup(sel);   // at once: the rest of the CTA learns the expert after a barrier
             }
+            issue_wave(sel);   // at once: the rest of the CTA learns the expert after a barrier
             if (blockIdx.x == 0 && lane < k) {
                 c.idx[lane] = my_e;
                 c.gates[lane] = p / zsum;
@@ -480,7 +511,6 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     }
     __syncthreads();
     ok = ok && s.ints[kIntAbort] == 0;
-    if (routed && ok && warp == 1) issue_down(s.ints[kIntSel]);
     if (routed && ok) wave_b = true;
     if (!routed && tid == 0) s.misc[kMiscGate] = s.misc[kMiscSgDot];
     if (blockIdx.x == 0 && tid == 32) {
