@@ -38,9 +38,14 @@
 // word that a CTA raises when one of its bounded waits runs out: the next call then zeroes the
 // accumulator and counters before anything is added, with no host intervention.
 //
-// GEMV arithmetic as in decode.cu: 4-bit codes enter the fp32 FMAs as subnormals (code * 2^-149),
-// the activations of each 64-column group are pre-scaled by a power of two, the scale is applied
-// once per (row, half group) and the bias as b * (sum of the half group's activations).
+// GEMV arithmetic: fp32 FMAs with fp16 multiplicands (fma.rn.f32.f16).  Each pair of 4-bit codes
+// is masked out of its packed word straight into the two halves of a 32-bit register, where it
+// reads as two fp16 subnormals (q * 2^-24, or q * 2^-20 for the upper nibble of a byte); the
+// activations are staged once per call as fp16, each 64-column group scaled by a power of two
+// (stage_f16), so every product is exact in fp32 and the sums are fp32.  The scale is applied once
+// per (row, half group) and the bias as b * (sum of the half group's staged activations).  x is
+// bf16, so staging it is exact (down to 2^-27 of its group's largest value); act is rounded to
+// fp16, as on the prefill path.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -53,15 +58,6 @@ constexpr int kDWarps = kDThreads / 32;
 constexpr int kMaxRouterRows = 4;
 constexpr int kMaxDM = 12;           // down blocks per CTA (H / 256)
 constexpr int kMaxChunkBlocks = 8;   // gate/up blocks per landing chunk
-
-__device__ __forceinline__ float pow2f(int n) { return __int_as_float((127 + n) << 23); }
-__device__ __forceinline__ int group_exponent(float m) {
-    int e = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
-    return max(-126, min(100, e));
-}
-// position of element e8 (0..7 of an 8-column word) in the order the code bytes come out:
-// (word & 0x0F0F0F0F) yields columns {0,4,1,5}, ((word >> 4) & 0x0F0F0F0F) columns {2,6,3,7}
-__device__ __forceinline__ int slot_of(int e8) { return (e8 >> 2) | ((e8 & 3) << 1); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -85,38 +81,53 @@ __device__ __forceinline__ uint32_t ord_key(float v) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// {a.x * b.x + c.x, a.y * b.y + c.y} in one packed fp32 FMA (sm_100), rounded once each, subnormal
-// operands kept (no .ftz): two of the GEMV's weight x activation products per instruction
-__device__ __forceinline__ float2 ffma2_keep_subnormal(float2 a, float2 b, float2 c) {
-    unsigned long long d;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
-        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
-        : "=l"(d)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-    return r;
+// {acc.x + c.lo * x.lo, acc.y + c.hi * x.hi}: fp32 FMAs with fp16 multiplicands (the product of
+// two fp16 values is exact in fp32, so each is rounded once, in the sum); the 4-bit codes enter as
+// fp16 subnormals, kept as such (no .ftz)
+__device__ __forceinline__ float2 fma_f16pair(uint32_t c2, uint32_t x2, float2 acc) {
+    float2 d;
+    asm("{\n\t.reg .b16 cl, ch, xl, xh;\n\tmov.b32 {cl, ch}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, cl, xl, %4;\n\tfma.rn.f32.f16 %1, ch, xh, %5;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "r"(c2), "r"(x2), "f"(acc.x), "f"(acc.y));
+    return d;
 }
 
-__device__ __forceinline__ float code_f(uint32_t m, uint32_t sel) { return __uint_as_float(__byte_perm(m, 0u, sel)); }
-
-// sum over the 32 columns of one half group: codes c (4 words), activations v in slot order
-__device__ __forceinline__ float dot32(const uint4& c, const float* v) {
+// Sum over the 32 columns of one half group: codes c (4 words of 8 nibbles), activations xv (32
+// fp16 in column order, 8 per uint4).  Nibbles of a word, low bit first, hold columns
+// 0 2 4 6 1 3 5 7, so the 16-bit halves of (w & 0x000F000F) are columns (0, 1) as q * 2^-24,
+// of (w & 0x00F000F0) columns (2, 3) as q * 2^-20, and the same masks of w >> 8 columns (4, 5)
+// and (6, 7): four ANDs and one shift per 8 columns.  The activations of pairs (2, 3) and (6, 7)
+// carry a further factor 2^-4 (stage_f16), so every product is q * x * 2^(A - 24) for the
+// group's A.
+__device__ __forceinline__ float dot32h(const uint4& c, const uint4* xv) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t m0 = w[i] & 0x0F0F0F0Fu;
-        const uint32_t m1 = (w[i] >> 4) & 0x0F0F0F0Fu;
-        const float4 x0 = *reinterpret_cast<const float4*>(v + 8 * i);
-        const float4 x1 = *reinterpret_cast<const float4*>(v + 8 * i + 4);
-        a = ffma2_keep_subnormal(make_float2(code_f(m0, 0x4440), code_f(m0, 0x4441)), make_float2(x0.x, x0.y), a);
-        b = ffma2_keep_subnormal(make_float2(code_f(m0, 0x4442), code_f(m0, 0x4443)), make_float2(x0.z, x0.w), b);
-        a = ffma2_keep_subnormal(make_float2(code_f(m1, 0x4440), code_f(m1, 0x4441)), make_float2(x1.x, x1.y), a);
-        b = ffma2_keep_subnormal(make_float2(code_f(m1, 0x4442), code_f(m1, 0x4443)), make_float2(x1.z, x1.w), b);
+        const uint4 xx = xv[i];
+        const uint32_t hi = w[i] >> 8;
+        a = fma_f16pair(w[i] & 0x000F000Fu, xx.x, a);
+        b = fma_f16pair(w[i] & 0x00F000F0u, xx.y, b);
+        a = fma_f16pair(hi & 0x000F000Fu, xx.z, a);
+        b = fma_f16pair(hi & 0x00F000F0u, xx.w, b);
     }
     return (a.x + a.y) + (b.x + b.y);
+}
+
+// Stages a lane's two consecutive columns (2 lane, 2 lane + 1) of a 64-column group for dot32h:
+// the group is scaled by 2^A, A = 14 - (exponent of the group's largest |value| m), so that every
+// value is below 2^15 in magnitude; columns 2-3 and 6-7 of each 8 take a further 2^-4; the values
+// are rounded to fp16 (bf16 inputs stay exact down to 2^-27 of the group's largest).  Returns the
+// two fp16 values; *rounded receives their sum as the GEMV sees them (unscaled, for the bias
+// term) and *undo the factor 2^(24 - A) that turns a dot32h sum into the plain dot.
+__device__ __forceinline__ uint32_t stage_f16(float a0, float a1, int lane, float m, float* rounded, float* undo) {
+    const int e = max(-100, min(100, (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127));
+    const int A = 14 - e - ((lane & 1) ? 4 : 0);
+    const __half2 h = __floats2half2_rn(a0 * __int_as_float((127 + A) << 23), a1 * __int_as_float((127 + A) << 23));
+    *rounded = (__low2float(h) + __high2float(h)) * __int_as_float((127 - A) << 23);
+    *undo = __int_as_float((127 + 10 + e) << 23);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // One comparator of the descending sort of a lane's (key, expert) pairs: the larger key first,
@@ -188,13 +199,13 @@ struct Smem {
     float* rrow;       // [R][H]      router rows of this CTA (routed units)
     float* sgw;        // [H]         shared-expert gate vector (shared units and CTA 0)
     float* xraw;       // [H]         x in fp32
-    float* xs;         // [H]         x pre-scaled per 64-column group, slot order
-    float* xsum;       // [H/32]      sum of x over each half group
-    float* xsc;        // [H/64]      2^(149-K) per group
+    uint32_t* xh;      // [H/2]       x as fp16 pairs, scaled per 64-column group (stage_f16)
+    float* xsum;       // [H/32]      sum of the staged x over each half group, unscaled
+    float* xsc;        // [H/64]      2^(24-A) per group (stage_f16)
     float* part;       // [4][128]    gate/up partial row sums (block parity x column half)
     float* mine;       // [128]       this CTA's gate/up row sums over its input-column half
     float* peer;       // [128]       the partner's, written by the partner
-    float* act;        // [64]        act of the slice, pre-scaled, slot order
+    uint32_t* act;     // [32]        act of the slice as fp16 pairs (stage_f16)
     float* misc;       // [8]         asum[2], asc, gate, shared-gate dot, logits reduction ...
     float* ydn;        // [2][DM*128] down partial sums by column half
     float* logit;      // [256]
@@ -210,14 +221,14 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const DecodeGeom& g) {
     s.rrow = reinterpret_cast<float*>(base + g.off_rrow);
     s.sgw = reinterpret_cast<float*>(base + g.off_sgw);
     s.xraw = reinterpret_cast<float*>(base + g.off_xraw);
-    s.xs = reinterpret_cast<float*>(base + g.off_xs);
+    s.xh = reinterpret_cast<uint32_t*>(base + g.off_xs);
     s.xsum = reinterpret_cast<float*>(base + g.off_xsum);
     s.xsc = reinterpret_cast<float*>(base + g.off_xsc);
     s.part = reinterpret_cast<float*>(base + g.off_part);
     s.mine = s.part + 4 * 128;
     s.peer = s.mine + 128;
-    s.act = s.peer + 128;
-    s.misc = s.act + 64;
+    s.act = reinterpret_cast<uint32_t*>(s.peer + 128);
+    s.misc = s.peer + 128 + 64;
     s.ydn = reinterpret_cast<float*>(base + g.off_ydn);
     s.logit = reinterpret_cast<float*>(base + g.off_logit);
     s.red = s.logit + 256;
@@ -410,14 +421,11 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     for (int grp = g.KH * (int)r + warp; grp < g.KH * ((int)r + 1); grp += kDWarps) {
         const float a0 = s.xraw[64 * grp + 2 * lane], a1 = s.xraw[64 * grp + 2 * lane + 1];
         const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(a0), fabsf(a1)))));
-        const float hs = half_warp_sum(a0 + a1);
-        const int K = 125 - group_exponent(m);
-        const float f1 = pow2f(K / 2), f2 = pow2f(K - K / 2);
-        const int e0 = 2 * lane, e1 = 2 * lane + 1;
-        s.xs[64 * grp + (e0 & ~7) + slot_of(e0 & 7)] = a0 * f1 * f2;
-        s.xs[64 * grp + (e1 & ~7) + slot_of(e1 & 7)] = a1 * f1 * f2;
+        float rsum, undo;
+        s.xh[32 * grp + lane] = stage_f16(a0, a1, lane, m, &rsum, &undo);
+        const float hs = half_warp_sum(rsum);
         if ((lane & 15) == 0) s.xsum[2 * grp + (lane >> 4)] = hs;
-        if (lane == 0) s.xsc[grp] = pow2f(149 - K);
+        if (lane == 0) s.xsc[grp] = undo;
     }
     if (ok && (routed || dirty) && warp == 0) {
         // every router word of this call: relaxed polls (each word carries its data; no load is
@@ -537,7 +545,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                     const uint8_t* blk = s.wgu + (size_t)b * kBlockBytes;
                     const uint4 cw = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
                     const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
-                    const float P = dot32(cw, s.xs + 64 * kc + 32 * hh);
+                    const float P = dot32h(cw, reinterpret_cast<const uint4*>(s.xh + 32 * kc + 16 * hh));
                     const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
                     const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
                     acc += sc * (P * s.xsc[kc]) + bi * s.xsum[2 * kc + hh];
@@ -571,16 +579,11 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
             a[u] = G * U / (1.f + expf(-G));
         }
         const float m = warp_max(fmaxf(fabsf(a[0]), fabsf(a[1])));
-        const float hs = half_warp_sum(a[0] + a[1]);
-        const int K = 125 - group_exponent(m);
-        const float f1 = pow2f(K / 2), f2 = pow2f(K - K / 2);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int i = 2 * lane + u;
-            s.act[(i & ~7) + slot_of(i & 7)] = a[u] * f1 * f2;
-        }
+        float rsum, undo;
+        s.act[lane] = stage_f16(a[0], a[1], lane, m, &rsum, &undo);
+        const float hs = half_warp_sum(rsum);
         if ((lane & 15) == 0) s.misc[kMiscAsum0 + (lane >> 4)] = hs;
-        if (lane == 0) s.misc[kMiscAsc] = pow2f(149 - K);
+        if (lane == 0) s.misc[kMiscAsc] = undo;
     }
     bool dok = ok;
     if (ok) dok = wait_bar(bar_d, 0);
@@ -588,9 +591,9 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
 
     // ---- 5. down GEMV: DM output m-tiles x 128 rows x this slice's 64 columns
     if (ok) {
-        float4 av[8];
+        uint4 av[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) av[i] = reinterpret_cast<const float4*>(s.act + 32 * hh)[i];
+        for (int i = 0; i < 4; ++i) av[i] = reinterpret_cast<const uint4*>(s.act + 16 * hh)[i];
         const float asc = s.misc[kMiscAsc], asum = s.misc[kMiscAsum0 + hh];
         // this thread's (up to kMaxDM / 2) blocks: every shared-memory load first, then the math
         uint4 cw[kMaxDM / 2];
@@ -608,7 +611,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         for (int i = 0; i < kMaxDM / 2; ++i) {
             const int b = par + 2 * i;
             if (b < g.DM) {
-                const float P = dot32(cw[i], reinterpret_cast<const float*>(av));
+                const float P = dot32h(cw[i], av);
                 const float sc = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
                 const float bi = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
                 s.ydn[hh * g.DM * 128 + b * 128 + row] = sc * (P * asc) + bi * asum;
