@@ -58,6 +58,8 @@ constexpr int kDWarps = kDThreads / 32;
 constexpr int kMaxRouterRows = 4;
 constexpr int kMaxDM = 12;           // down blocks per CTA (H / 256)
 constexpr int kMaxChunkBlocks = 8;   // gate/up blocks per landing chunk
+constexpr int kPollWarps = 3;        // warps polling the router words, staggered
+constexpr int kPollStaggerCycles = 500;
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -210,7 +212,7 @@ struct Smem {
     float* ydn;        // [2][DM*128] down partial sums by column half
     float* logit;      // [256]
     float* red;        // [kDWarps][kMaxRouterRows + 1] per-warp partial dots
-    int* ints;         // [16]        flags: abort, dirty, sel expert, chunk flags follow
+    int* ints;         // [kNumInts]  flags: abort, dirty, sel expert, tag, chunk flags, poll winner
     uint64_t* bars;    // bar_r, bar_d, bar_x, bar_g[0..3]
 };
 
@@ -237,7 +239,8 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const DecodeGeom& g) {
     return s;
 }
 
-enum { kIntAbort = 0, kIntDirty = 1, kIntSel = 2, kIntTag = 3, kIntFlags = 4 };   // ints[4 + b]: chunk b finalised here
+enum { kIntAbort = 0, kIntDirty = 1, kIntSel = 2, kIntTag = 3, kIntFlags = 4,   // ints[4 + b]: chunk b finalised here
+       kIntPolled = 4 + kMaxDM, kNumInts = 4 + kMaxDM + 4 };
 enum { kMiscAsum0 = 0, kMiscAsum1 = 1, kMiscAsc = 2, kMiscGate = 3, kMiscSgDot = 4 };
 
 __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, DecodeGeom g) {
@@ -266,6 +269,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         fence_mbar_init();
         mbar_arrive_expect_tx(bar_x, 128 * sizeof(float));   // before the partner can send (cluster barrier 1)
         s.ints[kIntAbort] = 0;
+        s.ints[kIntPolled] = 0;
     }
     cluster_arrive_relaxed();   // (1) this CTA has started; waited on before the first remote store
     __syncthreads();
@@ -427,11 +431,19 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         if ((lane & 15) == 0) s.xsum[2 * grp + (lane >> 4)] = hs;
         if (lane == 0) s.xsc[grp] = undo;
     }
-    if (ok && (routed || dirty) && warp == 0) {
+    if (ok && (routed || dirty) && (warp & 3) == 0 && warp < 4 * kPollWarps) {
         // every router word of this call: relaxed polls (each word carries its data; no load is
-        // left in flight when the loop ends)
+        // left in flight when the loop ends).  kPollWarps warps poll, their rounds staggered by a
+        // fraction of a round trip, so the last word is seen sooner after it lands; the first
+        // warp to see them all wins (shared-memory flag) and goes on, the others stop.
+        const int pw = warp >> 2;
+        if (pw > 0) {
+            const long long c0 = clock64();
+            while (clock64() - c0 < (long long)pw * kPollStaggerCycles) {}
+        }
         uint32_t key[8], idx[8];
         float lg[8];
+        bool lost = false;
         const unsigned long long t0 = globaltimer_ns();
         while (true) {
             unsigned long long cur[8];
@@ -445,13 +457,23 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                 lg[i] = (e < E && f == f) ? f : -INFINITY;
                 if (e < E && (uint32_t)(cur[i] >> 32) != tag) all = false;
             }
-            if (__all_sync(0xffffffffu, all)) break;
+            if (__all_sync(0xffffffffu, all)) {
+                int won = 0;
+                if (lane == 0) won = atomicCAS(&s.ints[kIntPolled], 0, 1) == 0;
+                lost = __shfl_sync(0xffffffffu, won, 0) == 0;
+                break;
+            }
+            if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.ints[kIntPolled]), 0) != 0) {
+                lost = true;   // another polling warp has them
+                break;
+            }
             if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {   // one decision for the warp
                 ok = false;
                 break;
             }
         }
         ok = __all_sync(0xffffffffu, ok);
+        if (lost) goto polled;
         if (dirty) fence_acq_rel_gpu();   // every routed CTA's zeroing precedes what follows
         if (ok && routed) {
             // top k by logit, ties to the lower expert index: each lane sorts its 8 (key, expert)
@@ -517,6 +539,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         }
         if (lane == 0) s.ints[kIntAbort] = ok ? 0 : 1;
     }
+polled:
     __syncthreads();
     ok = ok && s.ints[kIntAbort] == 0;
     if (routed && ok) wave_b = true;
@@ -691,7 +714,7 @@ bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeo
     g.off_xsc = o; o = al(o + sizeof(float) * (size_t)(H / 64));
     g.off_part = o; o = al(o + sizeof(float) * (4 * 128 + 128 + 128 + 64 + 8));
     g.off_ydn = o; o = al(o + sizeof(float) * 2 * (size_t)g.DM * 128);
-    g.off_logit = o; o = al(o + sizeof(float) * (256 + kDWarps * (kMaxRouterRows + 1)) + sizeof(int) * 16);
+    g.off_logit = o; o = al(o + sizeof(float) * (256 + kDWarps * (kMaxRouterRows + 1)) + sizeof(int) * kNumInts);
     g.off_bars = o; o = al(o + sizeof(uint64_t) * 7);
     g.smem = (int)o;
     if (g.smem > 227 * 1024) return false;
