@@ -148,9 +148,9 @@ Layout make_layout(const moe_config& c) {
     L.o_stage_x = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
     L.o_stage_out = take(sizeof(uint16_t) * (size_t)L.Tm * L.H);
     L.o_dfz_ticket = take(sizeof(unsigned long long));
-    L.o_dfz_slots = take(sizeof(unsigned long long) * (size_t)L.E);
-    L.o_dfz_outacc = take(sizeof(float) * (size_t)L.H);
-    L.o_dfz_cnt = take(sizeof(unsigned) * (size_t)(L.H / 128));
+    L.o_dfz_slots = take(sizeof(unsigned long long) * kDecodeFusedMaxT * (size_t)L.E);
+    L.o_dfz_outacc = take(sizeof(float) * kDecodeFusedMaxT * (size_t)L.H);
+    L.o_dfz_cnt = take(sizeof(unsigned) * kDecodeFusedMaxT * (size_t)(L.H / 128));
     L.o_dfz_dirty = take(sizeof(unsigned));
     L.ws_bytes = o;
     return L;
@@ -250,7 +250,8 @@ struct moe_handle {
     CUtensorMap amap_gu{}, amap_dn{};
     // batch-1 decode: the fused kernel's geometry, when the shape and the device allow it
     bool fused_ok = false;
-    DecodeGeom dgeom{};
+    DecodeGeom dgeom{};     // one token per launch
+    DecodeGeom dgeom_m{};   // 1 .. kDecodeFusedMaxT tokens per launch
 };
 
 namespace {
@@ -278,14 +279,11 @@ int check_call(moe_handle* h, const void* x, int32_t T, const void* out, bool ne
 
 bool use_decode(const moe_handle* h, int T) { return T <= h->cfg.decode_max_tokens; }
 
-// Decode calls of at most this many tokens run the single-token fused kernel once per token.
-// Measured per layer call in a 40-layer graph on one B200: fused 16.8 us per token; the
-// multi-kernel GEMV chain 59.9 / 75.0 / 98.9 us at T = 2 / 4 / 8; so per-token launches win up
-// to T = 4 (~67 us) and lose from T = 5 on.
-constexpr int kFusedDecodeMaxT = 4;
+// Decode calls of at most kDecodeFusedMaxT tokens run the fused kernel, one launch for all of
+// them; larger decode calls run the multi-kernel GEMV chain.
 
-// The fused kernel serves T == 1 when the shape fits its geometry and all of its clusters can be
-// resident at once (decided at create); otherwise the multi-kernel GEMV chain does.
+// The fused kernel serves T <= kDecodeFusedMaxT when the shape fits its geometry and all of its
+// clusters can be resident at once (decided at create); otherwise the multi-kernel GEMV chain does.
 bool fused_decode_ok(const moe_handle* h) { return h->fused_ok && !(h->cfg.flags & MOE_FLAG_DECODE_UNFUSED); }
 
 // Profiling: one event before the first kernel of a call and one after each kernel.
@@ -448,7 +446,8 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_hist, 0, sizeof(int) * (size_t)L.nblk_max * L.E, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_status, 0, sizeof(uint32_t) * 4, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_ticket, 0, sizeof(unsigned long long), st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_slots, 0, sizeof(unsigned long long) * (size_t)L.E, st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(h->ws + L.o_dfz_slots, 0, sizeof(unsigned long long) * kDecodeFusedMaxT * (size_t)L.E, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_dirty, 0x01, sizeof(unsigned), st);
     } else {
         e = cudaMemsetAsync(h->ws, 0, L.ws_bytes, st);
@@ -546,12 +545,15 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.dfz.cnt = reinterpret_cast<unsigned*>(ws + L.o_dfz_cnt);
     c.dfz.dirty = reinterpret_cast<unsigned*>(ws + L.o_dfz_dirty);
 
-    if (experts && router && decode_fused_geometry(L.H, L.I, L.E, L.k, cfg->has_shared, &h->dgeom)) {
-        int nclusters = 0;
+    if (experts && router && decode_fused_geometry(L.H, L.I, L.E, L.k, cfg->has_shared, 1, &h->dgeom) &&
+        decode_fused_geometry(L.H, L.I, L.E, L.k, cfg->has_shared, kDecodeFusedMaxT, &h->dgeom_m)) {
+        int n1 = 0, nm = 0;
         e = decode_fused_prepare(h->dgeom);
-        if (e == cudaSuccess) e = decode_fused_max_clusters(h->dgeom, &nclusters);
+        if (e == cudaSuccess) e = decode_fused_prepare(h->dgeom_m);
+        if (e == cudaSuccess) e = decode_fused_max_clusters(h->dgeom, &n1);
+        if (e == cudaSuccess) e = decode_fused_max_clusters(h->dgeom_m, &nm);
         if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "decode kernel set-up: %s", cudaGetErrorString(e)));
-        h->fused_ok = nclusters >= h->dgeom.units;
+        h->fused_ok = n1 >= h->dgeom.units && nm >= h->dgeom_m.units;
     }
 
     for (int hs = 0; hs < 3 && rc == MOE_OK; ++hs) {
@@ -595,17 +597,9 @@ int moe_forward(moe_handle* h, const uint16_t* x, int32_t T, uint16_t* out, void
     const bool decode = use_decode(h, T);
     const Ctx c = make_ctx(h, T, x, out, decode);
     Prof pf(h, st);
-    if (decode && T <= kFusedDecodeMaxT && fused_decode_ok(h)) {
-        // one launch of the single-token kernel per token (each a programmatic dependent of the
-        // last): for up to kFusedDecodeMaxT tokens this is faster than the multi-kernel chain
-        for (int t = 0; t < T; ++t) {
-            Ctx ct = c;
-            ct.T = 1;
-            ct.x = x + (size_t)t * h->L.H;
-            ct.out = out + (size_t)t * h->L.H;
-            MOE_LAUNCH("moe.decode_fused", launch_decode_fused(ct, h->dgeom, st));
-            pf.mark(9);
-        }
+    if (decode && T <= kDecodeFusedMaxT && fused_decode_ok(h)) {
+        MOE_LAUNCH("moe.decode_fused", launch_decode_fused(c, T == 1 ? h->dgeom : h->dgeom_m, st));
+        pf.mark(9);
         return MOE_OK;
     }
     rc = enqueue_routing(h, pf, c, decode, st);

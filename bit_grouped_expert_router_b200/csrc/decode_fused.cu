@@ -1,4 +1,5 @@
-// decode_fused.cu -- batch-1 decode of one MoE layer in a single kernel of CTA pairs.
+// decode_fused.cu -- decode of up to kDecodeFusedMaxT tokens through one MoE layer in a single
+// kernel of CTA pairs.
 //
 // A decode token moves ~18 MB (router 2 MiB + 9 experts x 1.69 MiB): about 2.8 us of HBM time,
 // so what decides the layer's time is how many dependent memory round trips lie on its critical
@@ -30,7 +31,11 @@
 //      row accumulator (vector reductions in L2); per 128-row chunk an arrival counter finds the
 //      last of the units, which rounds the chunk to bf16, writes it and re-zeroes the chunk's
 //      accumulator and counter (self-cleaning, no memset).
-// The shared-expert pairs never wait for routing.
+// The shared-expert pairs never wait for routing.  With T > 1 tokens every step keeps per-token
+// state (x, router words, selection, accumulators, counters); a routed unit runs steps 4-5 once
+// per token for the token's j-th expert, and its gate/up and down buffers take the next token's
+// expert as soon as the current token has read them, so that stream overlaps the current token's
+// exchange, act and down GEMV; the shared unit loads its weights once for all tokens.
 //
 // Call state lives in the workspace: a ticket counter every CTA increments at start (call number
 // = ticket / CTAs per call, so the router words of an earlier or abandoned call never carry the
@@ -58,7 +63,6 @@ constexpr int kDWarps = kDThreads / 32;
 constexpr int kMaxRouterRows = 4;
 constexpr int kMaxDM = 12;           // down blocks per CTA (H / 256)
 constexpr int kMaxChunkBlocks = 8;   // gate/up blocks per landing chunk
-constexpr int kPollWarps = 3;        // warps polling the router words, staggered
 constexpr int kPollStaggerCycles = 500;
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -195,59 +199,72 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
 }
 
 // Shared-memory carve-up (byte offsets, computed on the host from DecodeGeom and checked there).
+// Per-token arrays hold TM tokens.
 struct Smem {
-    uint8_t* wgu;      // [KH][4608]  gate/up blocks: this unit's m-tile, input-column half r
-    uint8_t* wdn;      // [DM][4608]  down blocks: k-step mt of the CTA's DM output m-tiles
+    uint8_t* wgu;      // [nslots][cblk][4608] gate/up chunk buffers (this unit's m-tile, column half r)
+    uint8_t* wdn;      // [1 or 2][DM][4608] down blocks: k-step mt of the CTA's DM output m-tiles
+                       //             (two buffers when TM > 1, by token parity)
     float* rrow;       // [R][H]      router rows of this CTA (routed units)
     float* sgw;        // [H]         shared-expert gate vector (shared units and CTA 0)
-    float* xraw;       // [H]         x in fp32
-    uint32_t* xh;      // [H/2]       x as fp16 pairs, scaled per 64-column group (stage_f16)
-    float* xsum;       // [H/32]      sum of the staged x over each half group, unscaled
-    float* xsc;        // [H/64]      2^(24-A) per group (stage_f16)
+    uint16_t* xraw;    // [T][H]      x as given (bf16)
+    uint32_t* xh;      // [T][H/2]    x as fp16 pairs, scaled per 64-column group (stage_f16)
+    float* xsum;       // [T][H/32]   sum of the staged x over each half group, unscaled
+    float* xsc;        // [T][H/64]   2^(24-A) per group (stage_f16)
     float* part;       // [4][128]    gate/up partial row sums (block parity x column half)
     float* mine;       // [128]       this CTA's gate/up row sums over its input-column half
-    float* peer;       // [128]       the partner's, written by the partner
+    float* peer;       // [2][128]    the partner's, written by the partner (by token parity)
     uint32_t* act;     // [32]        act of the slice as fp16 pairs (stage_f16)
-    float* misc;       // [8]         asum[2], asc, gate, shared-gate dot, logits reduction ...
+    float* misc;       // [16]        asum[2], asc; gate of token t at 4 + t; shared gate at 8 + t
     float* ydn;        // [2][DM*128] down partial sums by column half
-    float* logit;      // [256]
-    float* red;        // [kDWarps][kMaxRouterRows + 1] per-warp partial dots
-    int* ints;         // [kNumInts]  flags: abort, dirty, sel expert, tag, chunk flags, poll winner
-    uint64_t* bars;    // bar_r, bar_d, bar_x, bar_g[0..3]
+    float* red;        // [kDWarps][T][kMaxRouterRows + 1] per-warp partial dots (+ shared gate)
+    int* ints;         // [kNumInts]  flags, see below
+    uint64_t* bars;    // bar_r, bar_d[2], bar_x[2], bar_g[nslots]
 };
 
+template <int TM>
 __device__ __forceinline__ Smem carve(uint8_t* base, const DecodeGeom& g) {
     Smem s;
     s.wgu = base + g.off_wgu;
     s.wdn = base + g.off_wdn;
     s.rrow = reinterpret_cast<float*>(base + g.off_rrow);
     s.sgw = reinterpret_cast<float*>(base + g.off_sgw);
-    s.xraw = reinterpret_cast<float*>(base + g.off_xraw);
+    s.xraw = reinterpret_cast<uint16_t*>(base + g.off_xraw);
     s.xh = reinterpret_cast<uint32_t*>(base + g.off_xs);
     s.xsum = reinterpret_cast<float*>(base + g.off_xsum);
     s.xsc = reinterpret_cast<float*>(base + g.off_xsc);
     s.part = reinterpret_cast<float*>(base + g.off_part);
     s.mine = s.part + 4 * 128;
     s.peer = s.mine + 128;
-    s.act = reinterpret_cast<uint32_t*>(s.peer + 128);
-    s.misc = s.peer + 128 + 64;
+    s.act = reinterpret_cast<uint32_t*>(s.peer + 2 * 128);
+    s.misc = s.peer + 2 * 128 + 64;
     s.ydn = reinterpret_cast<float*>(base + g.off_ydn);
-    s.logit = reinterpret_cast<float*>(base + g.off_logit);
-    s.red = s.logit + 256;
-    s.ints = reinterpret_cast<int*>(s.red + kDWarps * (kMaxRouterRows + 1));
+    s.red = reinterpret_cast<float*>(base + g.off_logit);
+    s.ints = reinterpret_cast<int*>(s.red + kDWarps * TM * (kMaxRouterRows + 1));
     s.bars = reinterpret_cast<uint64_t*>(base + g.off_bars);
     return s;
 }
 
-enum { kIntAbort = 0, kIntDirty = 1, kIntSel = 2, kIntTag = 3, kIntFlags = 4,   // ints[4 + b]: chunk b finalised here
-       kIntPolled = 4 + kMaxDM, kNumInts = 4 + kMaxDM + 4 };
-enum { kMiscAsum0 = 0, kMiscAsum1 = 1, kMiscAsc = 2, kMiscGate = 3, kMiscSgDot = 4 };
+// ints: abort, dirty word, call tag, the selected expert of token t, the poll winner of token t,
+// copy waves issued into each gate/up chunk buffer and into each down buffer, and per (token,
+// chunk) whether this CTA finalises it
+constexpr int kMaxSlots = 8;
+enum {
+    kIntAbort = 0, kIntDirty = 1, kIntTag = 2, kIntSel = 3, kIntPolled = kIntSel + kDecodeFusedMaxT,
+    kIntWavesG = kIntPolled + kDecodeFusedMaxT, kIntWavesD = kIntWavesG + kMaxSlots,
+    kIntFlags = kIntWavesD + 2, kNumInts = kIntFlags + kDecodeFusedMaxT * kMaxDM
+};
+enum { kMiscAsum0 = 0, kMiscAsum1 = 1, kMiscAsc = 2, kMiscGate = 4, kMiscSg = 8 };
+constexpr int kRedStride = kMaxRouterRows + 1;   // per (warp, token): router rows, then the shared-gate dot
 
+// TM: the most tokens a launch serves (1: the single-token form, whose loops and per-token
+// registers collapse; kDecodeFusedMaxT: 1..kDecodeFusedMaxT tokens)
+template <int TM>
 __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, DecodeGeom g) {
+    constexpr int kPollWarps = TM == 1 ? 3 : 4;   // warps polling the router words (by token, then staggered)
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    const Smem s = carve(smem_raw, g);
+    const Smem s = carve<TM>(smem_raw, g);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = c.H, E = c.E, k = c.k;
+    const int H = c.H, E = c.E, k = c.k, T = TM == 1 ? 1 : c.T;
     const int KSg = H / 64, MTd = H / 128, KSd = c.I / 64;
     const uint32_t r = cluster_ctarank();
     const int q = blockIdx.x >> 1;                      // work unit = cluster
@@ -256,63 +273,52 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     const int mt = routed ? q % g.MTg : q - k * g.MTg;  // 64-column slice of I
     const int cr = blockIdx.x;                          // routed CTA index (routed units come first)
     uint64_t* bar_r = s.bars;       // router rows and the shared-gate vector landed
-    uint64_t* bar_d = s.bars + 1;   // down blocks landed
-    uint64_t* bar_x = s.bars + 2;   // the partner's gate/up sums landed (st.async from the partner)
-    uint64_t* bar_g = s.bars + 3;   // gate/up chunks landed
+    constexpr int kDSlots = TM > 1 ? 2 : 1;
+    uint64_t* bar_d = s.bars + 1;   // [kDSlots] down blocks landed (one phase per fill)
+    uint64_t* bar_x = s.bars + 3;   // [2] the partner's gate/up sums landed, by token parity
+    uint64_t* bar_g = s.bars + 5;   // [nslots] gate/up chunk buffers landed (one phase per fill)
     const bool need_sg = c.has_shared && (!routed || blockIdx.x == 0);
     int nrows = 0;   // router rows of this CTA
     if (routed)
         for (int i = 0; i < g.R; ++i) nrows += (cr + g.NR * i < E) ? 1 : 0;
 
     if (tid == 0) {
-        for (int i = 0; i < 3 + g.nch; ++i) mbar_init(&s.bars[i], 1);
+        for (int i = 0; i < 5 + g.nslots; ++i) mbar_init(&s.bars[i], 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_x, 128 * sizeof(float));   // before the partner can send (cluster barrier 1)
+        // exchange rounds 0 and 1, armed before the partner can send (cluster barrier 1)
+        mbar_arrive_expect_tx(&bar_x[0], 128 * sizeof(float));
+        if (T > 1) mbar_arrive_expect_tx(&bar_x[1], 128 * sizeof(float));
         s.ints[kIntAbort] = 0;
-        s.ints[kIntPolled] = 0;
+        for (int t = 0; t < kDecodeFusedMaxT; ++t) s.ints[kIntPolled + t] = 0;
+        for (int sl = 0; sl < kMaxSlots; ++sl) s.ints[kIntWavesG + sl] = (!routed && sl < g.nch) ? 1 : 0;
+        s.ints[kIntWavesD] = routed ? 0 : 1;
+        s.ints[kIntWavesD + 1] = 0;
     }
     cluster_arrive_relaxed();   // (1) this CTA has started; waited on before the first remote store
     __syncthreads();
 
     // ---- 1. weights that do not depend on x (nothing written by an earlier kernel is read yet)
-    // this unit's copies for expert e: the gate/up half in nch chunks (one thread), and the DM
-    // down blocks (one per lane of a warp, after lane 0 has set the barrier's byte count)
-    auto issue_gateup = [&](int e) {
-        const uint8_t* gu = c.w_gu + ((size_t)(e * g.MTg + mt) * KSg + (size_t)g.KH * r) * kBlockBytes;
-        for (int ch = 0; ch < g.nch; ++ch) {
-            const int b0 = ch * g.KH / g.nch, b1 = (ch + 1) * g.KH / g.nch;
-            mbar_arrive_expect_tx(&bar_g[ch], (uint32_t)((b1 - b0) * kBlockBytes));
-            bulk_g2s(s.wgu + (size_t)b0 * kBlockBytes, gu + (size_t)b0 * kBlockBytes, (uint32_t)((b1 - b0) * kBlockBytes),
-                     &bar_g[ch]);
-        }
+    // this unit's copies for expert e: the gate/up half in nch chunks (one thread, or one lane
+    // per chunk), and the DM down blocks (one per lane of a warp, after lane 0 has set the
+    // barrier's byte count).  A copy costs its issuing thread ~290 cycles, so a wave on the
+    // critical path is issued one copy per lane.
+    auto issue_gateup_chunk = [&](int e, int ch, int slot) {   // chunk ch of expert e into buffer slot
+        const uint8_t* gu = c.w_gu + ((size_t)(e * g.MTg + mt) * KSg + (size_t)g.KH * r + (size_t)ch * g.cblk) * kBlockBytes;
+        mbar_arrive_expect_tx(&bar_g[slot], (uint32_t)(g.cblk * kBlockBytes));
+        bulk_g2s(s.wgu + (size_t)slot * g.cblk * kBlockBytes, gu, (uint32_t)(g.cblk * kBlockBytes), &bar_g[slot]);
+        if (routed) ++s.ints[kIntWavesG + slot];   // one issuing thread per buffer at a time
     };
-    auto issue_down = [&](int e) {   // called by a whole warp
-        if (lane == 0) mbar_arrive_expect_tx(bar_d, (uint32_t)(g.DM * kBlockBytes));
+    auto issue_down = [&](int e, int dslot) {   // called by a whole warp
+        uint64_t* bd = &bar_d[dslot];
+        uint8_t* dst = s.wdn + (size_t)dslot * g.DM * kBlockBytes;
+        if (lane == 0) mbar_arrive_expect_tx(bd, (uint32_t)(g.DM * kBlockBytes));
         __syncwarp();
         for (int b = lane; b < g.DM; b += 32) {
             const int mtd = g.DM * (int)r + b;
-            bulk_g2s(s.wdn + (size_t)b * kBlockBytes, c.w_dn + ((size_t)(e * MTd + mtd) * KSd + mt) * kBlockBytes,
-                     kBlockBytes, bar_d);
+            bulk_g2s(dst + (size_t)b * kBlockBytes, c.w_dn + ((size_t)(e * MTd + mtd) * KSd + mt) * kBlockBytes,
+                     kBlockBytes, bd);
         }
-    };
-    // the routed unit's whole wave from the warp that picked the expert, one copy per lane (a
-    // bulk copy costs its issuing thread ~290 cycles, so one lane per copy issues them at once):
-    // lanes 0 .. nch-1 a gate/up chunk each, lanes 16 .. 16 + DM - 1 a down block each
-    auto issue_wave = [&](int e) {   // called by a whole warp
-        if (lane < g.nch) {
-            const uint8_t* gu = c.w_gu + ((size_t)(e * g.MTg + mt) * KSg + (size_t)g.KH * r) * kBlockBytes;
-            const int b0 = lane * g.KH / g.nch, b1 = (lane + 1) * g.KH / g.nch;
-            mbar_arrive_expect_tx(&bar_g[lane], (uint32_t)((b1 - b0) * kBlockBytes));
-            bulk_g2s(s.wgu + (size_t)b0 * kBlockBytes, gu + (size_t)b0 * kBlockBytes, (uint32_t)((b1 - b0) * kBlockBytes),
-                     &bar_g[lane]);
-        }
-        if (lane == 16) mbar_arrive_expect_tx(bar_d, (uint32_t)(g.DM * kBlockBytes));
-        __syncwarp();
-        if (lane >= 16 && lane - 16 < g.DM) {
-            const int b = lane - 16, mtd = g.DM * (int)r + b;
-            bulk_g2s(s.wdn + (size_t)b * kBlockBytes, c.w_dn + ((size_t)(e * MTd + mtd) * KSd + mt) * kBlockBytes,
-                     kBlockBytes, bar_d);
-        }
+        if (lane == 0 && routed) ++s.ints[kIntWavesD + dslot];
     };
     const bool need_r = nrows > 0 || need_sg;
     if (need_r && warp == 2 && lane == 0) {
@@ -322,26 +328,18 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                      bar_r);
         if (need_sg) bulk_g2s(s.sgw, c.sgw, (uint32_t)(H * sizeof(float)), bar_r);
     }
-    if (!routed) {   // the shared expert is group E
-        if (warp == 0 && lane == 0) issue_gateup(E);
-        if (warp == 1) issue_down(E);
+    if (!routed) {   // the shared expert is group E, the same for every token: one wave
+        if (warp == 0 && lane < g.nch) issue_gateup_chunk(E, lane, lane);
+        if (warp == 1) issue_down(E, 0);
     }
     const float my_bias = (tid < nrows) ? c.rbias[cr + g.NR * tid] : 0.f;
-    bool wave_b = !routed;   // this CTA's unit copies are in flight (drained before exit)
 
     // ---- 2. from here on x and the workspace are read: wait for the previous grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // x: 16-byte loads by the first H/8 threads; the call ticket and the dirty word are fetched
-    // by the last two warps at the same time (the tag is only needed at the router publish)
-    for (int i = tid; i < H / 8; i += kDThreads) {
-        const uint4 raw = reinterpret_cast<const uint4*>(c.x)[i];
-        reinterpret_cast<float4*>(s.xraw)[2 * i] =
-            make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u), __uint_as_float(raw.y << 16),
-                        __uint_as_float(raw.y & 0xFFFF0000u));
-        reinterpret_cast<float4*>(s.xraw)[2 * i + 1] =
-            make_float4(__uint_as_float(raw.z << 16), __uint_as_float(raw.z & 0xFFFF0000u), __uint_as_float(raw.w << 16),
-                        __uint_as_float(raw.w & 0xFFFF0000u));
-    }
+    // x of the T tokens: 16-byte loads; the call ticket and the dirty word are fetched by the last
+    // two warps at the same time (the tag is only needed at the router publish)
+    for (int i = tid; i < T * H / 8; i += kDThreads)
+        reinterpret_cast<uint4*>(s.xraw)[i] = reinterpret_cast<const uint4*>(c.x)[i];
     if (tid == kDThreads - 64) {   // call tag: CTAs started before this one, over CTAs per call (+1)
         const unsigned long long ticket = atomicAdd(c.dfz.ticket, 1ull);
         s.ints[kIntTag] = (int)(uint32_t)(ticket / (unsigned long long)gridDim.x + 1ull);
@@ -350,41 +348,59 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     __syncthreads();
     const uint32_t tag = (uint32_t)s.ints[kIntTag];
     const bool dirty = s.ints[kIntDirty] != 0;
-    // a call after one that gave up part-way: the routed CTAs put the accumulator and the chunk
-    // counters back to zero (ordered before their router words by a fence)
+    // a call after one that gave up part-way: the routed CTAs put the accumulators and the chunk
+    // counters of every token back to zero (ordered before their router words by a fence)
     if (dirty && routed) {
-        for (int i = cr * kDThreads + tid; i < H; i += g.NR * kDThreads) c.dfz.outacc[i] = 0.f;
-        for (int i = cr * kDThreads + tid; i < MTd; i += g.NR * kDThreads) c.dfz.cnt[i] = 0u;
+        for (int i = cr * kDThreads + tid; i < kDecodeFusedMaxT * H; i += g.NR * kDThreads) c.dfz.outacc[i] = 0.f;
+        for (int i = cr * kDThreads + tid; i < kDecodeFusedMaxT * MTd; i += g.NR * kDThreads) c.dfz.cnt[i] = 0u;
     }
 
-    // ---- 3. router logits and the shared gate sigmoid(x . w_sg) (the shared units' combine
-    // weight; CTA 0 also reports it)
+    // ---- 3. router logits and the shared gate sigmoid(x . w_sg) of every token (the shared
+    // units' combine weight; CTA 0 also reports it)
     bool ok = true;
     if (need_r) ok = wait_bar(bar_r, 0);
     {
-        float acc[kMaxRouterRows];
-        float d = 0.f;
+        float acc[TM][kMaxRouterRows];
+        float d[TM];
 #pragma unroll
-        for (int i = 0; i < kMaxRouterRows; ++i) acc[i] = 0.f;
+        for (int t = 0; t < TM; ++t) {
+            d[t] = 0.f;
+#pragma unroll
+            for (int i = 0; i < kMaxRouterRows; ++i) acc[t][i] = 0.f;
+        }
         if (ok) {
             for (int h = tid; h < H; h += kDThreads) {
-                const float xv = s.xraw[h];
+                float rv[kMaxRouterRows];
 #pragma unroll
-                for (int i = 0; i < kMaxRouterRows; ++i)
-                    if (i < nrows) acc[i] = fmaf(xv, s.rrow[(size_t)i * H + h], acc[i]);
-                if (need_sg) d = fmaf(xv, s.sgw[h], d);
+                for (int i = 0; i < kMaxRouterRows; ++i) rv[i] = i < nrows ? s.rrow[(size_t)i * H + h] : 0.f;
+                const float sv = need_sg ? s.sgw[h] : 0.f;
+#pragma unroll
+                for (int t = 0; t < TM; ++t) {
+                    if (t < T) {
+                        const float xv = __uint_as_float((uint32_t)s.xraw[(size_t)t * H + h] << 16);
+#pragma unroll
+                        for (int i = 0; i < kMaxRouterRows; ++i)
+                            if (i < nrows) acc[t][i] = fmaf(xv, rv[i], acc[t][i]);
+                        if (need_sg) d[t] = fmaf(xv, sv, d[t]);
+                    }
+                }
             }
         }
 #pragma unroll
-        for (int i = 0; i < kMaxRouterRows; ++i) {
-            if (i < nrows) {   // uniform across the CTA
-                const float v = warp_sum(acc[i]);
-                if (lane == 0) s.red[kDWarps + warp * kMaxRouterRows + i] = v;
+        for (int t = 0; t < TM; ++t) {
+            if (t < T) {   // uniform across the CTA
+#pragma unroll
+                for (int i = 0; i < kMaxRouterRows; ++i) {
+                    if (i < nrows) {
+                        const float v = warp_sum(acc[t][i]);
+                        if (lane == 0) s.red[(warp * TM + t) * kRedStride + i] = v;
+                    }
+                }
+                if (need_sg) {
+                    const float v = warp_sum(d[t]);
+                    if (lane == 0) s.red[(warp * TM + t) * kRedStride + kMaxRouterRows] = v;
+                }
             }
-        }
-        if (need_sg) {
-            d = warp_sum(d);
-            if (lane == 0) s.red[warp] = d;
         }
     }
     if (__syncthreads_or(!ok)) {
@@ -394,53 +410,54 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
             atomicOr(c.dfz.dirty, 1u);
         }
     }
-    if (routed && ok && warp == 0) {
-        // the per-warp partial dots of each router row, summed across warp 0's lanes
-        float zr[kMaxRouterRows];
+    if (routed && ok && warp == 0 && lane < T * nrows) {
+        // lane (t, i) sums router row i's per-warp partial dots of token t (all loads first)
+        const int t = lane / nrows, i = lane - t * nrows;
+        float pv[kDWarps];
 #pragma unroll
-        for (int i = 0; i < kMaxRouterRows; ++i) {
-            zr[i] = (lane < kDWarps && i < nrows) ? s.red[kDWarps + lane * kMaxRouterRows + i] : 0.f;
-            zr[i] = warp_sum(zr[i]);
-        }
+        for (int w = 0; w < kDWarps; ++w) pv[w] = s.red[(w * TM + t) * kRedStride + i];
         float z = 0.f;
 #pragma unroll
-        for (int i = 0; i < kMaxRouterRows; ++i)
-            if (lane == i) z = zr[i];
-        z += my_bias;
-        if (lane < nrows) {
-            const int e = cr + g.NR * lane;
-            const bool stall = (c.flags & 0x100u) && cr == 0 && tag == 1u;   // test only: first call withholds
-            // the word carries its own data; after a failed call it must also follow this CTA's zeroing
-            if (dirty) fence_acq_rel_gpu();
-            if (!stall) st_relaxed_u64(c.dfz.slots + e, ((unsigned long long)tag << 32) | __float_as_uint(z));
-        }
+        for (int w = 0; w < kDWarps; ++w) z += pv[w];
+        z += __shfl_sync((1u << (T * nrows)) - 1u, my_bias, i);
+        const int e = cr + g.NR * i;
+        const bool stall = (c.flags & 0x100u) && cr == 0 && tag == 1u;   // test only: first call withholds
+        // the word carries its own data; after a failed call it must also follow this CTA's zeroing
+        if (dirty) fence_acq_rel_gpu();
+        if (!stall) st_relaxed_u64(c.dfz.slots + (size_t)t * E + e, ((unsigned long long)tag << 32) | __float_as_uint(z));
     }
-    if (need_sg && tid == 32) {
+    if (need_sg && tid >= 32 && tid < 32 + T) {
+        const int t = tid - 32;
         float zz = 0.f;
-        for (int w = 0; w < kDWarps; ++w) zz += s.red[w];
-        s.misc[kMiscSgDot] = 1.f / (1.f + expf(-zz));
+        for (int w = 0; w < kDWarps; ++w) zz += s.red[(w * TM + t) * kRedStride + kMaxRouterRows];
+        s.misc[kMiscSg + t] = 1.f / (1.f + expf(-zz));
     }
-    // per-group scaling of the input-column half this CTA's gate/up blocks cover (only the gate/up
-    // GEMV reads it, so it follows the router publish)
-    for (int grp = g.KH * (int)r + warp; grp < g.KH * ((int)r + 1); grp += kDWarps) {
-        const float a0 = s.xraw[64 * grp + 2 * lane], a1 = s.xraw[64 * grp + 2 * lane + 1];
+    // per-group scaling of x over the input-column half this CTA's gate/up blocks cover, every
+    // token (only the gate/up GEMV reads it, so it follows the router publish)
+    for (int p = warp; p < T * g.KH; p += kDWarps) {
+        const int t = p / g.KH, grp = g.KH * (int)r + (p - t * g.KH);
+        const uint32_t xw = reinterpret_cast<const uint32_t*>(s.xraw + (size_t)t * H)[32 * grp + lane];
+        const float a0 = __uint_as_float(xw << 16), a1 = __uint_as_float(xw & 0xFFFF0000u);
         const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(a0), fabsf(a1)))));
         float rsum, undo;
-        s.xh[32 * grp + lane] = stage_f16(a0, a1, lane, m, &rsum, &undo);
+        s.xh[(size_t)t * (H / 2) + 32 * grp + lane] = stage_f16(a0, a1, lane, m, &rsum, &undo);
         const float hs = half_warp_sum(rsum);
-        if ((lane & 15) == 0) s.xsum[2 * grp + (lane >> 4)] = hs;
-        if (lane == 0) s.xsc[grp] = undo;
+        if ((lane & 15) == 0) s.xsum[(size_t)t * (H / 32) + 2 * grp + (lane >> 4)] = hs;
+        if (lane == 0) s.xsc[(size_t)t * (H / 64) + grp] = undo;
     }
     if (ok && (routed || dirty) && (warp & 3) == 0 && warp < 4 * kPollWarps) {
         // every router word of this call: relaxed polls (each word carries its data; no load is
-        // left in flight when the loop ends).  kPollWarps warps poll, their rounds staggered by a
-        // fraction of a round trip, so the last word is seen sooner after it lands; the first
-        // warp to see them all wins (shared-memory flag) and goes on, the others stop.
+        // left in flight when the loop ends).  kPollWarps warps poll; warp pw takes token pw % T,
+        // several warps on one token staggered by a fraction of a round trip so the last word is
+        // seen sooner after it lands; the first to see a token's words wins it (shared-memory
+        // flag) and goes on, the others stop.
         const int pw = warp >> 2;
-        if (pw > 0) {
+        const int tk = pw % T;
+        if (pw >= T) {
             const long long c0 = clock64();
-            while (clock64() - c0 < (long long)pw * kPollStaggerCycles) {}
+            while (clock64() - c0 < (long long)(pw / T) * kPollStaggerCycles) {}
         }
+        const unsigned long long* words = c.dfz.slots + (size_t)tk * E;
         uint32_t key[8], idx[8];
         float lg[8];
         bool lost = false;
@@ -448,7 +465,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         while (true) {
             unsigned long long cur[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) cur[i] = (lane + 32 * i < E) ? ld_relaxed_u64(c.dfz.slots + lane + 32 * i) : 0ull;
+            for (int i = 0; i < 8; ++i) cur[i] = (lane + 32 * i < E) ? ld_relaxed_u64(words + lane + 32 * i) : 0ull;
             bool all = true;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -459,12 +476,12 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
             }
             if (__all_sync(0xffffffffu, all)) {
                 int won = 0;
-                if (lane == 0) won = atomicCAS(&s.ints[kIntPolled], 0, 1) == 0;
+                if (lane == 0) won = atomicCAS(&s.ints[kIntPolled + tk], 0, 1) == 0;
                 lost = __shfl_sync(0xffffffffu, won, 0) == 0;
                 break;
             }
-            if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.ints[kIntPolled]), 0) != 0) {
-                lost = true;   // another polling warp has them
+            if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.ints[kIntPolled + tk]), 0) != 0) {
+                lost = true;   // another polling warp has this token's words
                 break;
             }
             if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {   // one decision for the warp
@@ -524,162 +541,217 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
             const int sel = __shfl_sync(0xffffffffu, my_e, j);
             const float gsel = __shfl_sync(0xffffffffu, p, j) / zsum;
             if (lane == 0) {
-                s.ints[kIntSel] = sel;
-                s.misc[kMiscGate] = gsel;
+                s.ints[kIntSel + tk] = sel;
+                s.misc[kMiscGate + tk] = gsel;
             }
-            issue_wave(sel);   // at once: the rest of the CTA learns the expert after a barrier
+            if (tk == 0) {   // the first token's wave at once: lanes 0 .. nch-1 a gate/up chunk each,
+                             // lanes 16 .. 16 + DM - 1 a down block each
+                if (lane < g.nch) issue_gateup_chunk(sel, lane, lane);
+                if (lane == 16) mbar_arrive_expect_tx(bar_d, (uint32_t)(g.DM * kBlockBytes));
+                __syncwarp();
+                if (lane >= 16 && lane - 16 < g.DM) {
+                    const int b = lane - 16, mtd = g.DM * (int)r + b;
+                    bulk_g2s(s.wdn + (size_t)b * kBlockBytes,
+                             c.w_dn + ((size_t)(sel * MTd + mtd) * KSd + mt) * kBlockBytes, kBlockBytes, bar_d);
+                }
+                if (lane == 16) s.ints[kIntWavesD] = 1;
+            }
             if (blockIdx.x == 0 && lane < k) {
-                c.idx[lane] = my_e;
-                c.gates[lane] = p / zsum;
+                c.idx[(size_t)tk * k + lane] = my_e;
+                c.gates[(size_t)tk * k + lane] = p / zsum;
             }
         }
         if (lane == 0 && !ok) {
             set_status(c.status, MOE_STATUS_TIMEOUT);
             atomicOr(c.dfz.dirty, 1u);
         }
-        if (lane == 0) s.ints[kIntAbort] = ok ? 0 : 1;
+        if (lane == 0 && !ok) s.ints[kIntAbort] = 1;
     }
 polled:
     __syncthreads();
     ok = ok && s.ints[kIntAbort] == 0;
-    if (routed && ok) wave_b = true;
-    if (!routed && tid == 0) s.misc[kMiscGate] = s.misc[kMiscSgDot];
-    if (blockIdx.x == 0 && tid == 32) {
-        c.sg[0] = c.has_shared ? s.misc[kMiscSgDot] : 0.f;
-        if (ok && dirty) st_release_u32(c.dfz.dirty, 0u);   // every routed CTA has read it
+    if (TM > 1 && routed && ok && T > 1 && warp == 1) issue_down(s.ints[kIntSel + 1], 1);   // token 1's down blocks
+    if (!routed && tid < T) s.misc[kMiscGate + tid] = s.misc[kMiscSg + tid];
+    if (blockIdx.x == 0 && tid >= 32 && tid < 32 + T) {
+        c.sg[tid - 32] = c.has_shared ? s.misc[kMiscSg + tid - 32] : 0.f;
     }
+    if (blockIdx.x == 0 && tid == 64 && ok && dirty) st_release_u32(c.dfz.dirty, 0u);   // every routed CTA has read it
     // the next kernel in the stream may be scheduled from here on (it waits for this grid's
     // completion before it reads anything this grid writes)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    // ---- 4. gate/up GEMV over this CTA's input-column half, as the chunks land
+    // ---- 4./5. per token: gate/up GEMV as the chunks land, the pair's exchange, act, down GEMV,
+    // gated reductions into the token's fp32 row.  A routed unit's gate/up chunk buffers take the
+    // next token's expert once this token's GEMV has read them (the stream overlaps this token's
+    // exchange, act and down GEMV); with TM > 1 its down blocks alternate between two buffers, so
+    // the next token's are in flight before this token's down GEMV; the shared unit's weights
+    // serve every token.
     const int row = tid & 127, hh = (tid >> 7) & 1, par = tid >> 8;
-    float acc = 0.f;
-    bool wok = ok;
-    if (ok) {
-        for (int ch = 0; ch < g.nch; ++ch) {
-            if (!wait_bar(&bar_g[ch], 0)) { wok = false; break; }
-            const int b0 = ch * g.KH / g.nch, b1 = (ch + 1) * g.KH / g.nch;
+    unsigned arrivals[TM];   // counter values before this CTA's arrival (tid < DM)
 #pragma unroll
-            for (int i = 0; i < kMaxChunkBlocks / 2; ++i) {
-                const int b = b0 + par + 2 * i;
-                if (b < b1) {
-                    const int kc = g.KH * (int)r + b;   // 64-column group of x
-                    const uint8_t* blk = s.wgu + (size_t)b * kBlockBytes;
-                    const uint4 cw = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
-                    const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
-                    const float P = dot32h(cw, reinterpret_cast<const uint4*>(s.xh + 32 * kc + 16 * hh));
-                    const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
-                    const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
-                    acc += sc * (P * s.xsc[kc]) + bi * s.xsum[2 * kc + hh];
+    for (int t = 0; t < TM; ++t) arrivals[t] = 0u;
+    for (int t = 0; t < T; ++t) {
+        // this token's down blocks: buffer t % 2 (TM > 1) and that buffer's fill, or the shared
+        // unit's one fill
+        const int dslot = (TM > 1 && routed) ? (t & 1) : 0;
+        const uint32_t ph = routed ? (uint32_t)((TM > 1 ? t >> 1 : t) & 1) : 0u;
+        float acc = 0.f;
+        bool wok = ok;
+        if (ok) {
+            const uint32_t* xt = s.xh + (size_t)t * (H / 2);
+            for (int ch = 0; ch < g.nch; ++ch) {
+                // chunk number cs of the unit's gate/up stream, in buffer cs % nslots (the shared
+                // unit's chunks stay in buffers 0 .. nch-1 for every token)
+                const int cs = routed ? t * g.nch + ch : ch;
+                const int slot = cs % g.nslots;
+                if (!wait_bar(&bar_g[slot], (uint32_t)((cs / g.nslots) & 1))) { wok = false; break; }
+                const uint8_t* cbase = s.wgu + (size_t)slot * g.cblk * kBlockBytes;
+#pragma unroll
+                for (int i = 0; i < kMaxChunkBlocks / 2; ++i) {
+                    const int b = par + 2 * i;
+                    if (b < g.cblk) {
+                        const int kc = g.KH * (int)r + ch * g.cblk + b;   // 64-column group of x
+                        const uint8_t* blk = cbase + (size_t)b * kBlockBytes;
+                        const uint4 cw = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
+                        const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+                        const float P = dot32h(cw, reinterpret_cast<const uint4*>(xt + 32 * kc + 16 * hh));
+                        const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+                        const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
+                        acc += sc * (P * s.xsc[(size_t)t * (H / 64) + kc]) +
+                               bi * s.xsum[(size_t)t * (H / 32) + 2 * kc + hh];
+                    }
                 }
             }
         }
-    }
-    s.part[(par * 2 + hh) * 128 + row] = acc;
-    if (__syncthreads_or(!wok)) ok = false;
-    if (ok && tid < 128) s.mine[tid] = (s.part[tid] + s.part[128 + tid]) + (s.part[256 + tid] + s.part[384 + tid]);
-    cluster_wait();   // (1) the partner has started (its exchange mbarrier expects our 512 bytes)
-    __syncthreads();
-    // the pair's exchange: this CTA's 128 row sums go into the partner's shared memory with
-    // asynchronous remote stores that complete the partner's mbarrier; each CTA waits on its own.
-    // A CTA that gave up still waits for its partner's sums (bounded), so neither exits while the
-    // other may still be writing into it.
-    if (ok && tid < 32)
-        st_async_peer_v4(s.peer + 4 * tid, bar_x, r ^ 1u, reinterpret_cast<const float4*>(s.mine)[tid]);
-    if (!wait_bar(bar_x, 0)) ok = false;
-    if (__syncthreads_or(!ok)) ok = false;
+        s.part[(par * 2 + hh) * 128 + row] = acc;
+        if (__syncthreads_or(!wok)) ok = false;
+        // the gate/up buffers are read: the next token's expert streams into them, one chunk per lane
+        if (TM > 1 && routed && ok && t + 1 < T && warp == 0 && lane < g.nch)
+            issue_gateup_chunk(s.ints[kIntSel + t + 1], lane, lane);
+        if (ok && tid < 128) s.mine[tid] = (s.part[tid] + s.part[128 + tid]) + (s.part[256 + tid] + s.part[384 + tid]);
+        if (t == 0) cluster_wait();   // (1) the partner has started (its exchange mbarriers are armed)
+        __syncthreads();
+        // the pair's exchange, round t: this CTA's 128 row sums go into the partner's shared memory
+        // with asynchronous remote stores that complete the partner's mbarrier of this token
+        // parity; each CTA waits on its own.  Both CTAs take every round whatever their state
+        // (a CTA that gave up sends what it has), so neither exits while the other may still be
+        // writing into it, and no round waits for a partner that has left.
+        float* peer = s.peer + 128 * (t & 1);
+        uint64_t* bx = &bar_x[t & 1];
+        if (tid < 32) st_async_peer_v4(peer + 4 * tid, bx, r ^ 1u, reinterpret_cast<const float4*>(s.mine)[tid]);
+        if (!wait_bar(bx, (uint32_t)((t >> 1) & 1))) ok = false;
+        if (__syncthreads_or(!ok)) ok = false;
+        if (tid == 0 && t + 2 < T) mbar_arrive_expect_tx(bx, 128 * sizeof(float));   // round t + 2
 
-    // act = silu(G) * U for the slice's 64 columns: G and U of column i are rows 32(i/16) + i%16
-    // and 16 rows further of the interleaved m-tile; pre-scaled for the down GEMV
-    if (ok && warp == 0) {
-        float a[2];
+        // act = silu(G) * U for the slice's 64 columns: G and U of column i are rows 32(i/16) + i%16
+        // and 16 rows further of the interleaved m-tile; staged in fp16 for the down GEMV
+        if (ok && warp == 0) {
+            float a[2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int i = 2 * lane + u;
-            const int rg = 32 * (i >> 4) + (i & 15), ru = rg + 16;
-            const float G = s.mine[rg] + s.peer[rg], U = s.mine[ru] + s.peer[ru];
-            a[u] = G * U / (1.f + expf(-G));
+            for (int u = 0; u < 2; ++u) {
+                const int i = 2 * lane + u;
+                const int rg = 32 * (i >> 4) + (i & 15), ru = rg + 16;
+                const float G = s.mine[rg] + peer[rg], U = s.mine[ru] + peer[ru];
+                a[u] = G * U / (1.f + expf(-G));
+            }
+            const float m = warp_max(fmaxf(fabsf(a[0]), fabsf(a[1])));
+            float rsum, undo;
+            s.act[lane] = stage_f16(a[0], a[1], lane, m, &rsum, &undo);
+            const float hs = half_warp_sum(rsum);
+            if ((lane & 15) == 0) s.misc[kMiscAsum0 + (lane >> 4)] = hs;
+            if (lane == 0) s.misc[kMiscAsc] = undo;
         }
-        const float m = warp_max(fmaxf(fabsf(a[0]), fabsf(a[1])));
-        float rsum, undo;
-        s.act[lane] = stage_f16(a[0], a[1], lane, m, &rsum, &undo);
-        const float hs = half_warp_sum(rsum);
-        if ((lane & 15) == 0) s.misc[kMiscAsum0 + (lane >> 4)] = hs;
-        if (lane == 0) s.misc[kMiscAsc] = undo;
-    }
-    bool dok = ok;
-    if (ok) dok = wait_bar(bar_d, 0);
-    if (__syncthreads_or(!dok)) ok = false;
+        bool dok = ok;
+        if (ok) dok = wait_bar(&bar_d[dslot], ph);
+        if (__syncthreads_or(!dok)) ok = false;
 
-    // ---- 5. down GEMV: DM output m-tiles x 128 rows x this slice's 64 columns
-    if (ok) {
-        uint4 av[4];
+        // down GEMV: DM output m-tiles x 128 rows x this slice's 64 columns
+        if (ok) {
+            uint4 av[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) av[i] = reinterpret_cast<const uint4*>(s.act + 16 * hh)[i];
-        const float asc = s.misc[kMiscAsc], asum = s.misc[kMiscAsum0 + hh];
-        // this thread's (up to kMaxDM / 2) blocks: every shared-memory load first, then the math
-        uint4 cw[kMaxDM / 2];
-        uint32_t sb[kMaxDM / 2];
+            for (int i = 0; i < 4; ++i) av[i] = reinterpret_cast<const uint4*>(s.act + 16 * hh)[i];
+            const float asc = s.misc[kMiscAsc], asum = s.misc[kMiscAsum0 + hh];
+            // this thread's (up to kMaxDM / 2) blocks: every shared-memory load first, then the math
+            uint4 cw[kMaxDM / 2];
+            uint32_t sb[kMaxDM / 2];
 #pragma unroll
-        for (int i = 0; i < kMaxDM / 2; ++i) {
-            const int b = par + 2 * i;
-            if (b < g.DM) {
-                const uint8_t* blk = s.wdn + (size_t)b * kBlockBytes;
-                cw[i] = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
-                sb[i] = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+            for (int i = 0; i < kMaxDM / 2; ++i) {
+                const int b = par + 2 * i;
+                if (b < g.DM) {
+                    const uint8_t* blk = s.wdn + ((size_t)dslot * g.DM + b) * kBlockBytes;
+                    cw[i] = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
+                    sb[i] = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kMaxDM / 2; ++i) {
+                const int b = par + 2 * i;
+                if (b < g.DM) {
+                    const float P = dot32h(cw[i], av);
+                    const float sc = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
+                    const float bi = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
+                    s.ydn[hh * g.DM * 128 + b * 128 + row] = sc * (P * asc) + bi * asum;
+                }
             }
         }
-#pragma unroll
-        for (int i = 0; i < kMaxDM / 2; ++i) {
-            const int b = par + 2 * i;
-            if (b < g.DM) {
-                const float P = dot32h(cw[i], av);
-                const float sc = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
-                const float bi = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
-                s.ydn[hh * g.DM * 128 + b * 128 + row] = sc * (P * asc) + bi * asum;
+        __syncthreads();
+        // the down buffer is read: the expert of the token after next streams into it
+        if (TM > 1 && routed && ok && t + 2 < T && warp == 1) issue_down(s.ints[kIntSel + t + 2], dslot);
+        if (ok) {
+            const float gate = s.misc[kMiscGate + t];
+            const int nrow = g.DM * 128;
+            float* dst = c.dfz.outacc + (size_t)t * H + (size_t)g.DM * r * 128;
+            for (int i4 = tid; 4 * i4 < nrow; i4 += kDThreads) {
+                const float4 y0 = reinterpret_cast<const float4*>(s.ydn)[i4];
+                const float4 y1 = reinterpret_cast<const float4*>(s.ydn + nrow)[i4];
+                red_add_v4(dst + 4 * i4, (y0.x + y1.x) * gate, (y0.y + y1.y) * gate, (y0.z + y1.z) * gate,
+                           (y0.w + y1.w) * gate);
             }
         }
-    }
-    __syncthreads();
-    if (ok) {
-        const float gate = s.misc[kMiscGate];
-        const int nrow = g.DM * 128;
-        float* dst = c.dfz.outacc + (size_t)g.DM * r * 128;
-        for (int i4 = tid; 4 * i4 < nrow; i4 += kDThreads) {
-            const float4 y0 = reinterpret_cast<const float4*>(s.ydn)[i4];
-            const float4 y1 = reinterpret_cast<const float4*>(s.ydn + nrow)[i4];
-            red_add_v4(dst + 4 * i4, (y0.x + y1.x) * gate, (y0.y + y1.y) * gate, (y0.z + y1.z) * gate,
-                       (y0.w + y1.w) * gate);
+        __syncthreads();
+        // one arrival per 128-row chunk of this token; the counter values are read after the
+        // last token, so the round trip overlaps the next token's work
+        if (ok && tid < g.DM) {
+#pragma unroll
+            for (int u = 0; u < TM; ++u)
+                if (u == t) arrivals[u] = atom_add_acq_rel(c.dfz.cnt + (size_t)t * MTd + g.DM * (int)r + tid, 1u);
         }
     }
-    __syncthreads();
-    // one arrival per 128-row chunk; the last of the units finalises the chunk
+    // the last of the units to arrive at a (token, chunk) finalises it: bf16 out, accumulator and
+    // counter back to zero
     if (ok && tid < g.DM) {
-        const int mtd = g.DM * (int)r + tid;
-        const unsigned old = atom_add_acq_rel(c.dfz.cnt + mtd, 1u);
-        s.ints[kIntFlags + tid] = (old == (unsigned)(g.units - 1)) ? 1 : 0;
+#pragma unroll
+        for (int u = 0; u < TM; ++u)
+            if (u < T) s.ints[kIntFlags + u * kMaxDM + tid] = (arrivals[u] == (unsigned)(g.units - 1)) ? 1 : 0;
     }
     __syncthreads();
     if (ok) {
-        for (int i = tid; i < g.DM * 128; i += kDThreads) {
-            if (!s.ints[kIntFlags + (i >> 7)]) continue;
-            const size_t hrow = (size_t)g.DM * r * 128 + i;
-            const float v = atomicExch(c.dfz.outacc + hrow, 0.f);
-            c.out[hrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        for (int t = 0; t < T; ++t) {
+            for (int i = tid; i < g.DM * 128; i += kDThreads) {
+                if (!s.ints[kIntFlags + t * kMaxDM + (i >> 7)]) continue;
+                const size_t hrow = (size_t)g.DM * r * 128 + i;
+                const float v = atomicExch(c.dfz.outacc + (size_t)t * H + hrow, 0.f);
+                c.out[(size_t)t * H + hrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
+            if (tid < g.DM && s.ints[kIntFlags + t * kMaxDM + tid])
+                atomicExch(c.dfz.cnt + (size_t)t * MTd + g.DM * (int)r + tid, 0u);
         }
-        if (tid < g.DM && s.ints[kIntFlags + tid]) atomicExch(c.dfz.cnt + g.DM * (int)r + tid, 0u);
     }
     if (!ok && tid == 0) {
         set_status(c.status, MOE_STATUS_TIMEOUT);
         atomicOr(c.dfz.dirty, 1u);
     }
-    // nothing may still be landing in this CTA's shared memory when it exits
+    // nothing may still be landing in this CTA's shared memory when it exits: the last wave
+    // issued into each buffer has landed (earlier ones were waited for, or precede it)
     if (tid == 0) {
         if (need_r) mbar_drain(bar_r, 0);
-        if (wave_b) {
-            for (int ch = 0; ch < g.nch; ++ch) mbar_drain(&bar_g[ch], 0);
-            mbar_drain(bar_d, 0);
+        for (int sl = 0; sl < g.nslots; ++sl) {
+            const int wg = s.ints[kIntWavesG + sl];
+            if (wg > 0) mbar_drain(&bar_g[sl], (uint32_t)((wg - 1) & 1));
+        }
+        for (int ds = 0; ds < kDSlots; ++ds) {
+            const int wd = s.ints[kIntWavesD + ds];
+            if (wd > 0) mbar_drain(&bar_d[ds], (uint32_t)((wd - 1) & 1));
         }
     }
     __syncthreads();
@@ -689,9 +761,11 @@ polled:
 
 // Launch geometry of the fused kernel for a layer shape, or false when the shape does not fit it
 // (the multi-kernel GEMV chain then serves batch-1 decode).
-bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeom* out) {
+bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, int tm, DecodeGeom* out) {
     DecodeGeom g{};
     if (H % 256 != 0 || I % 64 != 0) return false;
+    if (tm != 1 && tm != kDecodeFusedMaxT) return false;
+    g.tm = tm;
     g.MTg = I / 64;
     g.units = (k + has_shared) * g.MTg;
     g.NR = 2 * k * g.MTg;
@@ -699,23 +773,28 @@ bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeo
     if (g.R > kMaxRouterRows) return false;
     g.KH = H / 128;
     g.nch = g.KH < 4 ? g.KH : 4;
+    if (g.KH % g.nch != 0) return false;
+    g.cblk = g.KH / g.nch;
+    if (g.cblk > kMaxChunkBlocks) return false;
+    g.nslots = g.nch;
+    if (g.nslots > kMaxSlots) return false;
     g.DM = H / 256;
     if (g.DM > kMaxDM) return false;   // also bounds the chunk flags in the ints area
-    if ((g.KH + g.nch - 1) / g.nch > kMaxChunkBlocks) return false;
     auto al = [](size_t v) { return (v + 127) / 128 * 128; };
+    const size_t TM = (size_t)tm;
     size_t o = 0;
-    g.off_wgu = o; o = al(o + (size_t)g.KH * kBlockBytes);
-    g.off_wdn = o; o = al(o + (size_t)g.DM * kBlockBytes);
+    g.off_wgu = o; o = al(o + (size_t)g.nslots * g.cblk * kBlockBytes);
+    g.off_wdn = o; o = al(o + (size_t)(tm > 1 ? 2 : 1) * g.DM * kBlockBytes);
     g.off_rrow = o; o = al(o + sizeof(float) * (size_t)g.R * H);
     g.off_sgw = o; o = al(o + sizeof(float) * (size_t)H);
-    g.off_xraw = o; o = al(o + sizeof(float) * (size_t)H);
-    g.off_xs = o; o = al(o + sizeof(float) * (size_t)H);
-    g.off_xsum = o; o = al(o + sizeof(float) * (size_t)(H / 32));
-    g.off_xsc = o; o = al(o + sizeof(float) * (size_t)(H / 64));
-    g.off_part = o; o = al(o + sizeof(float) * (4 * 128 + 128 + 128 + 64 + 8));
+    g.off_xraw = o; o = al(o + sizeof(uint16_t) * TM * H);
+    g.off_xs = o; o = al(o + sizeof(uint32_t) * TM * (H / 2));
+    g.off_xsum = o; o = al(o + sizeof(float) * TM * (H / 32));
+    g.off_xsc = o; o = al(o + sizeof(float) * TM * (H / 64));
+    g.off_part = o; o = al(o + sizeof(float) * (4 * 128 + 128 + 2 * 128 + 64 + 16));
     g.off_ydn = o; o = al(o + sizeof(float) * 2 * (size_t)g.DM * 128);
-    g.off_logit = o; o = al(o + sizeof(float) * (256 + kDWarps * (kMaxRouterRows + 1)) + sizeof(int) * kNumInts);
-    g.off_bars = o; o = al(o + sizeof(uint64_t) * 7);
+    g.off_logit = o; o = al(o + sizeof(float) * kDWarps * TM * kRedStride + sizeof(int) * kNumInts);
+    g.off_bars = o; o = al(o + sizeof(uint64_t) * (5 + (size_t)g.nslots));
     g.smem = (int)o;
     if (g.smem > 227 * 1024) return false;
     *out = g;
@@ -723,7 +802,9 @@ bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeo
 }
 
 cudaError_t decode_fused_prepare(const DecodeGeom& g) {
-    return cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem);
+    if (g.tm == 1) return cudaFuncSetAttribute(decode_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem);
+    return cudaFuncSetAttribute(decode_fused_kernel<kDecodeFusedMaxT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                g.smem);
 }
 
 // Clusters of the fused kernel that fit on the device at once (all must be resident together).
@@ -739,10 +820,13 @@ cudaError_t decode_fused_max_clusters(const DecodeGeom& g, int* n) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaOccupancyMaxActiveClusters(n, decode_fused_kernel, &cfg);
+    if (g.tm == 1) return cudaOccupancyMaxActiveClusters(n, decode_fused_kernel<1>, &cfg);
+    return cudaOccupancyMaxActiveClusters(n, decode_fused_kernel<kDecodeFusedMaxT>, &cfg);
 }
 
+// One launch for c.T tokens (1 <= c.T <= g.tm) with geometry g (decode_fused_geometry of g.tm).
 cudaError_t launch_decode_fused(const Ctx& c, const DecodeGeom& g, cudaStream_t st) {
+    if (c.T < 1 || c.T > g.tm) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * g.units);
     cfg.blockDim = dim3(kDThreads);
@@ -757,7 +841,8 @@ cudaError_t launch_decode_fused(const Ctx& c, const DecodeGeom& g, cudaStream_t 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, decode_fused_kernel, c, g);
+    if (g.tm == 1) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<1>, c, g);
+    return cudaLaunchKernelEx(&cfg, decode_fused_kernel<kDecodeFusedMaxT>, c, g);
 }
 
 }  // namespace moe

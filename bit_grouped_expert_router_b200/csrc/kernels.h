@@ -32,11 +32,14 @@ struct RepackArgs {
 };
 
 // Workspace of the fused batch-1 decode kernel (zero when the handle is created).
+// Tokens one launch of the fused decode kernel serves (its per-token buffers are sized for this).
+constexpr int kDecodeFusedMaxT = 4;
+
 struct DecodeFusedWs {
     unsigned long long* ticket;   // [1] CTAs started, over all calls (call number = ticket / CTAs per call)
-    unsigned long long* slots;    // [E] router logit of expert e as (call tag << 32) | fp32 bits
-    float* outacc;                // [H] fp32 output accumulator; zero between calls
-    unsigned* cnt;                // [H/128] unit arrivals per 128-row output chunk; zero between calls
+    unsigned long long* slots;    // [kDecodeFusedMaxT][E] router logit of (token, expert) as (call tag << 32) | fp32 bits
+    float* outacc;                // [kDecodeFusedMaxT][H] fp32 output accumulators; zero between calls
+    unsigned* cnt;                // [kDecodeFusedMaxT][H/128] unit arrivals per 128-row output chunk; zero between calls
     unsigned* dirty;              // [1] raised by a call that gave up part-way; the next call resets
 };
 
@@ -48,6 +51,9 @@ struct DecodeGeom {
     int R;        // router rows per routed CTA (ceil(E / NR))
     int KH;       // gate/up blocks per CTA (H / 128: one input-column half)
     int nch;      // landing chunks of the gate/up copy
+    int cblk;     // gate/up blocks per chunk (KH / nch)
+    int nslots;   // gate/up chunk buffers (nch)
+    int tm;       // the most tokens a launch with this geometry serves (1 or kDecodeFusedMaxT)
     int DM;       // down blocks per CTA (H / 256 output m-tiles)
     int smem;     // dynamic shared memory bytes
     size_t off_wgu, off_wdn, off_rrow, off_sgw, off_xraw, off_xs, off_xsum, off_xsc, off_part, off_ydn, off_logit, off_bars;
@@ -149,7 +155,8 @@ int gemm_tile_rows(int T, int k, int E);
 void set_last_error(const char* msg);
 
 // decode sparse GEMV
-bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, DecodeGeom* out);
+// tm: 1 (the single-token form) or kDecodeFusedMaxT (1..kDecodeFusedMaxT tokens per launch)
+bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, int tm, DecodeGeom* out);
 cudaError_t decode_fused_prepare(const DecodeGeom& g);
 cudaError_t decode_fused_max_clusters(const DecodeGeom& g, int* n);
 cudaError_t launch_decode_fused(const Ctx& c, const DecodeGeom& g, cudaStream_t st);

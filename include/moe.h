@@ -72,8 +72,8 @@ extern "C" {
 /* ---- configuration flags ---------------------------------------------------------------------- */
 #define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
 #define MOE_FLAG_DECODE_UNFUSED  0x2u  /* decode calls of T <= 4 tokens: use the multi-kernel
-                                          GEMV chain instead of the fused single-token kernel
-                                          (launched once per token) */
+                                          GEMV chain instead of the fused decode kernel (one
+                                          launch for all the call's tokens, up to 4) */
 #define MOE_FLAG_POISON_WORKSPACE 0x4u /* test aid: the handle's workspace starts filled with 0xFF
                                           bytes (NaN floats, -1 indices) instead of zeros, except
                                           the words the kernels count on starting at zero, so a
@@ -100,7 +100,7 @@ extern "C" {
                                           moe_route (and moe_combine_rows) only: the router of an
                                           expert-parallel layer whose experts live on other GPUs */
 #define MOE_FLAG_TEST_STALL      0x100u /* test only: the prefill producer withholds its loads on
-                                          every call, and the fused batch-1 decode kernel withholds
+                                          every call, and the fused decode kernel withholds
                                           one router result on the handle's first call, so bounded
                                           waits run out and the call reports
                                           MOE_ERR_DEVICE_TIMEOUT; nothing traps or hangs */
@@ -247,8 +247,8 @@ MOE_API int moe_debug_copy(moe_handle *h, int which, void *dst, size_t bytes, vo
  * device time in milliseconds (ms[MOE_PROF_SLOTS]) and the number of launches
  * (launches[MOE_PROF_SLOTS]), and clears the record.  Slots: 0 router logits, 1 top-k and gates,
  * 2 bucket scan, 3 scatter/gather, 4 gate/up grouped GEMM, 5 down grouped GEMM + combine,
- * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine, 9 fused batch-1 decode (the
- * whole layer in one kernel), 10 gather of token rows into bucket order.
+ * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine, 9 fused decode of up to 4 tokens
+ * (the whole layer in one kernel), 10 gather of token rows into bucket order.
  * Errors: INVALID_ARG, CUDA. */
 #define MOE_PROF_SLOTS 11
 MOE_API int moe_profile_enable(moe_handle *h, int enable);
