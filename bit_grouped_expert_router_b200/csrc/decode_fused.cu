@@ -605,21 +605,21 @@ polled:
                 const int cs = routed ? t * g.nch + ch : ch;
                 const int slot = cs % g.nslots;
                 if (!wait_bar(&bar_g[slot], (uint32_t)((cs / g.nslots) & 1))) { wok = false; break; }
-                const uint8_t* cbase = s.wgu + (size_t)slot * g.cblk * kBlockBytes;
-#pragma unroll
-                for (int i = 0; i < kMaxChunkBlocks / 2; ++i) {
-                    const int b = par + 2 * i;
-                    if (b < g.cblk) {
-                        const int kc = g.KH * (int)r + ch * g.cblk + b;   // 64-column group of x
-                        const uint8_t* blk = cbase + (size_t)b * kBlockBytes;
-                        const uint4 cw = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
-                        const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
-                        const float P = dot32h(cw, reinterpret_cast<const uint4*>(xt + 32 * kc + 16 * hh));
-                        const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
-                        const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
-                        acc += sc * (P * s.xsc[(size_t)t * (H / 64) + kc]) +
-                               bi * s.xsum[(size_t)t * (H / 32) + 2 * kc + hh];
-                    }
+                const uint8_t* cbase = s.wgu + (size_t)slot * g.cblk * kBlockBytes + hh * 2048 + row * 16;
+                const int kc0 = g.KH * (int)r + ch * g.cblk;   // first 64-column group of x in the chunk
+                const uint4* xc = reinterpret_cast<const uint4*>(xt + 32 * kc0 + 16 * hh);
+                const float* xscc = s.xsc + (size_t)t * (H / 64) + kc0;
+                const float* xsumc = s.xsum + (size_t)t * (H / 32) + 2 * kc0 + hh;
+#pragma unroll 2
+                for (int b = par; b < g.cblk; b += 2) {
+                    const uint8_t* blk = cbase + (size_t)b * kBlockBytes;
+                    const uint4 cw = *reinterpret_cast<const uint4*>(blk);
+                    const uint32_t sb =
+                        *reinterpret_cast<const uint32_t*>(blk - hh * 2048 - row * 16 + kBlockCodeBytes + row * 4);
+                    const float P = dot32h(cw, xc + 8 * b);
+                    const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+                    const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
+                    acc += sc * (P * xscc[b]) + bi * xsumc[2 * b];
                 }
             }
         }
