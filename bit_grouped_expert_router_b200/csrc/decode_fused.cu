@@ -386,19 +386,35 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                 }
             }
         }
+        if (TM == 1) {
+            // one token: the warp sums of every router row and of the shared-gate dot, their
+            // shuffle rounds interleaved (rows past nrows are zeros)
+            float v[kRedStride];
 #pragma unroll
-        for (int t = 0; t < TM; ++t) {
-            if (t < T) {   // uniform across the CTA
+            for (int i = 0; i < kMaxRouterRows; ++i) v[i] = acc[0][i];
+            v[kMaxRouterRows] = d[0];
 #pragma unroll
-                for (int i = 0; i < kMaxRouterRows; ++i) {
-                    if (i < nrows) {
-                        const float v = warp_sum(acc[t][i]);
-                        if (lane == 0) s.red[(warp * TM + t) * kRedStride + i] = v;
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int i = 0; i < kRedStride; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+            if (lane == 0)
+#pragma unroll
+                for (int i = 0; i < kRedStride; ++i) s.red[warp * kRedStride + i] = v[i];
+        } else {
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                if (t < T) {   // uniform across the CTA
+#pragma unroll
+                    for (int i = 0; i < kMaxRouterRows; ++i) {
+                        if (i < nrows) {
+                            const float v = warp_sum(acc[t][i]);
+                            if (lane == 0) s.red[(warp * TM + t) * kRedStride + i] = v;
+                        }
                     }
-                }
-                if (need_sg) {
-                    const float v = warp_sum(d[t]);
-                    if (lane == 0) s.red[(warp * TM + t) * kRedStride + kMaxRouterRows] = v;
+                    if (need_sg) {
+                        const float v = warp_sum(d[t]);
+                        if (lane == 0) s.red[(warp * TM + t) * kRedStride + kMaxRouterRows] = v;
+                    }
                 }
             }
         }
@@ -671,27 +687,18 @@ polled:
 #pragma unroll
             for (int i = 0; i < 4; ++i) av[i] = reinterpret_cast<const uint4*>(s.act + 16 * hh)[i];
             const float asc = s.misc[kMiscAsc], asum = s.misc[kMiscAsum0 + hh];
-            // this thread's (up to kMaxDM / 2) blocks: every shared-memory load first, then the math
-            uint4 cw[kMaxDM / 2];
-            uint32_t sb[kMaxDM / 2];
-#pragma unroll
-            for (int i = 0; i < kMaxDM / 2; ++i) {
-                const int b = par + 2 * i;
-                if (b < g.DM) {
-                    const uint8_t* blk = s.wdn + ((size_t)dslot * g.DM + b) * kBlockBytes;
-                    cw[i] = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
-                    sb[i] = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < kMaxDM / 2; ++i) {
-                const int b = par + 2 * i;
-                if (b < g.DM) {
-                    const float P = dot32h(cw[i], av);
-                    const float sc = __half2float(__ushort_as_half((unsigned short)(sb[i] & 0xFFFFu)));
-                    const float bi = __half2float(__ushort_as_half((unsigned short)(sb[i] >> 16)));
-                    s.ydn[hh * g.DM * 128 + b * 128 + row] = sc * (P * asc) + bi * asum;
-                }
+            // this thread's blocks b = par, par + 2, ... of the DM
+            const uint8_t* dbase = s.wdn + (size_t)dslot * g.DM * kBlockBytes;
+            float* yd = s.ydn + hh * g.DM * 128 + row;
+#pragma unroll 2
+            for (int b = par; b < g.DM; b += 2) {
+                const uint8_t* blk = dbase + (size_t)b * kBlockBytes;
+                const uint4 cw = *reinterpret_cast<const uint4*>(blk + hh * 2048 + row * 16);
+                const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+                const float P = dot32h(cw, av);
+                const float sc = __half2float(__ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+                const float bi = __half2float(__ushort_as_half((unsigned short)(sb >> 16)));
+                yd[b * 128] = sc * (P * asc) + bi * asum;
             }
         }
         __syncthreads();
