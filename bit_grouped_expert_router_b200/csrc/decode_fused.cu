@@ -202,8 +202,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
 // Per-token arrays hold TM tokens.
 struct Smem {
     uint8_t* wgu;      // [nslots][cblk][4608] gate/up chunk buffers (this unit's m-tile, column half r)
-    uint8_t* wdn;      // [1 or 2][DM][4608] down blocks: k-step mt of the CTA's DM output m-tiles
-                       //             (two buffers when TM > 1, by token parity)
+    uint8_t* wdn;      // [DM][4608]  down blocks: k-step mt of the CTA's DM output m-tiles
     float* rrow;       // [R][H]      router rows of this CTA (routed units)
     float* sgw;        // [H]         shared-expert gate vector (shared units and CTA 0)
     uint16_t* xraw;    // [T][H]      x as given (bf16)
@@ -214,7 +213,7 @@ struct Smem {
     float* mine;       // [128]       this CTA's gate/up row sums over its input-column half
     float* peer;       // [2][128]    the partner's, written by the partner (by token parity)
     uint32_t* act;     // [32]        act of the slice as fp16 pairs (stage_f16)
-    float* misc;       // [16]        asum[2], asc; gate of token t at 4 + t; shared gate at 8 + t
+    float* misc;       // [32]        asum[2], asc; gate of token t at 4 + t; shared gate at 4 + TM + t
     float* ydn;        // [2][DM*128] down partial sums by column half
     float* red;        // [kDWarps][T][kMaxRouterRows + 1] per-warp partial dots (+ shared gate)
     int* ints;         // [kNumInts]  flags, see below
@@ -236,7 +235,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const DecodeGeom& g) {
     s.mine = s.part + 4 * 128;
     s.peer = s.mine + 128;
     s.act = reinterpret_cast<uint32_t*>(s.peer + 2 * 128);
-    s.misc = s.peer + 2 * 128 + 64;
+    s.misc = s.peer + 2 * 128 + 64;   // [32]
     s.ydn = reinterpret_cast<float*>(base + g.off_ydn);
     s.red = reinterpret_cast<float*>(base + g.off_logit);
     s.ints = reinterpret_cast<int*>(s.red + kDWarps * TM * (kMaxRouterRows + 1));
@@ -253,14 +252,17 @@ enum {
     kIntWavesG = kIntPolled + kDecodeFusedMaxT, kIntWavesD = kIntWavesG + kMaxSlots,
     kIntFlags = kIntWavesD + 2, kNumInts = kIntFlags + kDecodeFusedMaxT * kMaxDM
 };
-enum { kMiscAsum0 = 0, kMiscAsum1 = 1, kMiscAsc = 2, kMiscGate = 4, kMiscSg = 8 };
+enum { kMiscAsum0 = 0, kMiscAsum1 = 1, kMiscAsc = 2, kMiscGate = 4, kMiscSg = 4 + kDecodeFusedMaxT };
+static_assert(kMiscSg + kDecodeFusedMaxT <= 32, "misc area");
 constexpr int kRedStride = kMaxRouterRows + 1;   // per (warp, token): router rows, then the shared-gate dot
 
 // TM: the most tokens a launch serves (1: the single-token form, whose loops and per-token
 // registers collapse; kDecodeFusedMaxT: 1..kDecodeFusedMaxT tokens)
 template <int TM>
 __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, DecodeGeom g) {
-    constexpr int kPollWarps = TM == 1 ? 3 : 4;   // warps polling the router words (by token, then staggered)
+    // warps polling the router words (every kPollStride-th warp; by token, then staggered)
+    constexpr int kPollWarps = TM == 1 ? 3 : kDecodeFusedMaxT;
+    constexpr int kPollStride = TM == 1 ? 4 : kDWarps / kDecodeFusedMaxT;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const Smem s = carve<TM>(smem_raw, g);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     const int mt = routed ? q % g.MTg : q - k * g.MTg;  // 64-column slice of I
     const int cr = blockIdx.x;                          // routed CTA index (routed units come first)
     uint64_t* bar_r = s.bars;       // router rows and the shared-gate vector landed
-    constexpr int kDSlots = TM > 1 ? 2 : 1;
+    constexpr int kDSlots = 1;
     uint64_t* bar_d = s.bars + 1;   // [kDSlots] down blocks landed (one phase per fill)
     uint64_t* bar_x = s.bars + 3;   // [2] the partner's gate/up sums landed, by token parity
     uint64_t* bar_g = s.bars + 5;   // [nslots] gate/up chunk buffers landed (one phase per fill)
@@ -359,14 +361,16 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
     // units' combine weight; CTA 0 also reports it)
     bool ok = true;
     if (need_r) ok = wait_bar(bar_r, 0);
-    {
-        float acc[TM][kMaxRouterRows];
-        float d[TM];
+    // tokens in passes of up to four (the per-thread partial sums live in registers)
+    constexpr int kTG = TM < 4 ? TM : 4;
+    for (int t0 = 0; t0 < T; t0 += kTG) {
+        float acc[kTG][kMaxRouterRows];
+        float d[kTG];
 #pragma unroll
-        for (int t = 0; t < TM; ++t) {
-            d[t] = 0.f;
+        for (int u = 0; u < kTG; ++u) {
+            d[u] = 0.f;
 #pragma unroll
-            for (int i = 0; i < kMaxRouterRows; ++i) acc[t][i] = 0.f;
+            for (int i = 0; i < kMaxRouterRows; ++i) acc[u][i] = 0.f;
         }
         if (ok) {
             for (int h = tid; h < H; h += kDThreads) {
@@ -375,13 +379,13 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                 for (int i = 0; i < kMaxRouterRows; ++i) rv[i] = i < nrows ? s.rrow[(size_t)i * H + h] : 0.f;
                 const float sv = need_sg ? s.sgw[h] : 0.f;
 #pragma unroll
-                for (int t = 0; t < TM; ++t) {
-                    if (t < T) {
-                        const float xv = __uint_as_float((uint32_t)s.xraw[(size_t)t * H + h] << 16);
+                for (int u = 0; u < kTG; ++u) {
+                    if (t0 + u < T) {
+                        const float xv = __uint_as_float((uint32_t)s.xraw[(size_t)(t0 + u) * H + h] << 16);
 #pragma unroll
                         for (int i = 0; i < kMaxRouterRows; ++i)
-                            if (i < nrows) acc[t][i] = fmaf(xv, rv[i], acc[t][i]);
-                        if (need_sg) d[t] = fmaf(xv, sv, d[t]);
+                            if (i < nrows) acc[u][i] = fmaf(xv, rv[i], acc[u][i]);
+                        if (need_sg) d[u] = fmaf(xv, sv, d[u]);
                     }
                 }
             }
@@ -402,17 +406,18 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
                 for (int i = 0; i < kRedStride; ++i) s.red[warp * kRedStride + i] = v[i];
         } else {
 #pragma unroll
-            for (int t = 0; t < TM; ++t) {
+            for (int u = 0; u < kTG; ++u) {
+                const int t = t0 + u;
                 if (t < T) {   // uniform across the CTA
 #pragma unroll
                     for (int i = 0; i < kMaxRouterRows; ++i) {
                         if (i < nrows) {
-                            const float v = warp_sum(acc[t][i]);
+                            const float v = warp_sum(acc[u][i]);
                             if (lane == 0) s.red[(warp * TM + t) * kRedStride + i] = v;
                         }
                     }
                     if (need_sg) {
-                        const float v = warp_sum(d[t]);
+                        const float v = warp_sum(d[u]);
                         if (lane == 0) s.red[(warp * TM + t) * kRedStride + kMaxRouterRows] = v;
                     }
                 }
@@ -435,7 +440,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         float z = 0.f;
 #pragma unroll
         for (int w = 0; w < kDWarps; ++w) z += pv[w];
-        z += __shfl_sync((1u << (T * nrows)) - 1u, my_bias, i);
+        z += __shfl_sync(T * nrows >= 32 ? 0xffffffffu : (1u << (T * nrows)) - 1u, my_bias, i);
         const int e = cr + g.NR * i;
         const bool stall = (c.flags & 0x100u) && cr == 0 && tag == 1u;   // test only: first call withholds
         // the word carries its own data; after a failed call it must also follow this CTA's zeroing
@@ -461,13 +466,13 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
         if ((lane & 15) == 0) s.xsum[(size_t)t * (H / 32) + 2 * grp + (lane >> 4)] = hs;
         if (lane == 0) s.xsc[(size_t)t * (H / 64) + grp] = undo;
     }
-    if (ok && (routed || dirty) && (warp & 3) == 0 && warp < 4 * kPollWarps) {
+    if (ok && (routed || dirty) && warp % kPollStride == 0 && warp < kPollStride * kPollWarps) {
         // every router word of this call: relaxed polls (each word carries its data; no load is
         // left in flight when the loop ends).  kPollWarps warps poll; warp pw takes token pw % T,
         // several warps on one token staggered by a fraction of a round trip so the last word is
         // seen sooner after it lands; the first to see a token's words wins it (shared-memory
         // flag) and goes on, the others stop.
-        const int pw = warp >> 2;
+        const int pw = warp / kPollStride;
         const int tk = pw % T;
         if (pw >= T) {
             const long long c0 = clock64();
@@ -586,7 +591,6 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(Ctx c, Decod
 polled:
     __syncthreads();
     ok = ok && s.ints[kIntAbort] == 0;
-    if (TM > 1 && routed && ok && T > 1 && warp == 1) issue_down(s.ints[kIntSel + 1], 1);   // token 1's down blocks
     if (!routed && tid < T) s.misc[kMiscGate + tid] = s.misc[kMiscSg + tid];
     if (blockIdx.x == 0 && tid >= 32 && tid < 32 + T) {
         c.sg[tid - 32] = c.has_shared ? s.misc[kMiscSg + tid - 32] : 0.f;
@@ -599,18 +603,16 @@ polled:
     // ---- 4./5. per token: gate/up GEMV as the chunks land, the pair's exchange, act, down GEMV,
     // gated reductions into the token's fp32 row.  A routed unit's gate/up chunk buffers take the
     // next token's expert once this token's GEMV has read them (the stream overlaps this token's
-    // exchange, act and down GEMV); with TM > 1 its down blocks alternate between two buffers, so
-    // the next token's are in flight before this token's down GEMV; the shared unit's weights
-    // serve every token.
+    // exchange, act and down GEMV), and its down buffer the next token's expert once this
+    // token's down GEMV has read it; the shared unit's weights serve every token.
     const int row = tid & 127, hh = (tid >> 7) & 1, par = tid >> 8;
     unsigned arrivals[TM];   // counter values before this CTA's arrival (tid < DM)
 #pragma unroll
     for (int t = 0; t < TM; ++t) arrivals[t] = 0u;
     for (int t = 0; t < T; ++t) {
-        // this token's down blocks: buffer t % 2 (TM > 1) and that buffer's fill, or the shared
-        // unit's one fill
-        const int dslot = (TM > 1 && routed) ? (t & 1) : 0;
-        const uint32_t ph = routed ? (uint32_t)((TM > 1 ? t >> 1 : t) & 1) : 0u;
+        // this token's fill of the down buffer (the shared unit's one fill serves every token)
+        const int dslot = 0;
+        const uint32_t ph = routed ? (uint32_t)(t & 1) : 0u;
         float acc = 0.f;
         bool wok = ok;
         if (ok) {
@@ -702,8 +704,8 @@ polled:
             }
         }
         __syncthreads();
-        // the down buffer is read: the expert of the token after next streams into it
-        if (TM > 1 && routed && ok && t + 2 < T && warp == 1) issue_down(s.ints[kIntSel + t + 2], dslot);
+        // the down buffer is read: the next token's expert streams into it
+        if (TM > 1 && routed && ok && t + 1 < T && warp == 1) issue_down(s.ints[kIntSel + t + 1], dslot);
         if (ok) {
             const float gate = s.misc[kMiscGate + t];
             const int nrow = g.DM * 128;
@@ -791,14 +793,14 @@ bool decode_fused_geometry(int H, int I, int E, int k, int has_shared, int tm, D
     const size_t TM = (size_t)tm;
     size_t o = 0;
     g.off_wgu = o; o = al(o + (size_t)g.nslots * g.cblk * kBlockBytes);
-    g.off_wdn = o; o = al(o + (size_t)(tm > 1 ? 2 : 1) * g.DM * kBlockBytes);
+    g.off_wdn = o; o = al(o + (size_t)g.DM * kBlockBytes);
     g.off_rrow = o; o = al(o + sizeof(float) * (size_t)g.R * H);
     g.off_sgw = o; o = al(o + sizeof(float) * (size_t)H);
     g.off_xraw = o; o = al(o + sizeof(uint16_t) * TM * H);
     g.off_xs = o; o = al(o + sizeof(uint32_t) * TM * (H / 2));
     g.off_xsum = o; o = al(o + sizeof(float) * TM * (H / 32));
     g.off_xsc = o; o = al(o + sizeof(float) * TM * (H / 64));
-    g.off_part = o; o = al(o + sizeof(float) * (4 * 128 + 128 + 2 * 128 + 64 + 16));
+    g.off_part = o; o = al(o + sizeof(float) * (4 * 128 + 128 + 2 * 128 + 64 + 32));
     g.off_ydn = o; o = al(o + sizeof(float) * 2 * (size_t)g.DM * 128);
     g.off_logit = o; o = al(o + sizeof(float) * kDWarps * TM * kRedStride + sizeof(int) * kNumInts);
     g.off_bars = o; o = al(o + sizeof(uint64_t) * (5 + (size_t)g.nslots));

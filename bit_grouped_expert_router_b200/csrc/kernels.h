@@ -33,7 +33,7 @@ struct RepackArgs {
 
 // Workspace of the fused batch-1 decode kernel (zero when the handle is created).
 // Tokens one launch of the fused decode kernel serves (its per-token buffers are sized for this).
-constexpr int kDecodeFusedMaxT = 4;
+constexpr int kDecodeFusedMaxT = 8;
 
 struct DecodeFusedWs {
     unsigned long long* ticket;   // [1] CTAs started, over all calls (call number = ticket / CTAs per call)

@@ -71,9 +71,9 @@ extern "C" {
 
 /* ---- configuration flags ---------------------------------------------------------------------- */
 #define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
-#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* decode calls of T <= 4 tokens: use the multi-kernel
+#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* decode calls of T <= 8 tokens: use the multi-kernel
                                           GEMV chain instead of the fused decode kernel (one
-                                          launch for all the call's tokens, up to 4) */
+                                          launch for all the call's tokens, up to 8) */
 #define MOE_FLAG_POISON_WORKSPACE 0x4u /* test aid: the handle's workspace starts filled with 0xFF
                                           bytes (NaN floats, -1 indices) instead of zeros, except
                                           the words the kernels count on starting at zero, so a
@@ -247,7 +247,7 @@ MOE_API int moe_debug_copy(moe_handle *h, int which, void *dst, size_t bytes, vo
  * device time in milliseconds (ms[MOE_PROF_SLOTS]) and the number of launches
  * (launches[MOE_PROF_SLOTS]), and clears the record.  Slots: 0 router logits, 1 top-k and gates,
  * 2 bucket scan, 3 scatter/gather, 4 gate/up grouped GEMM, 5 down grouped GEMM + combine,
- * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine, 9 fused decode of up to 4 tokens
+ * 6 finalize, 7 decode gate/up GEMV, 8 decode down GEMV + combine, 9 fused decode of up to 8 tokens
  * (the whole layer in one kernel), 10 gather of token rows into bucket order.
  * Errors: INVALID_ARG, CUDA. */
 #define MOE_PROF_SLOTS 11

@@ -207,10 +207,12 @@ def test_full_decode_workload(layer_idx):
     layer = _layer(w, shape, max_tokens=4096, decode_max_tokens=16)
     _route_check(layer, ol, x[:1], shape)
     print("decode T=1", _forward_check(layer, ol, x[:1]))
-    print("decode T=2 (fused kernel per token)", _forward_check(layer, ol, x[:2]))
-    print("decode T=4 (fused kernel per token)", _forward_check(layer, ol, x[:4]))
-    print("decode T=5 (GEMV chain)", _forward_check(layer, ol, x[:5]))
-    print("decode T=16", _forward_check(layer, ol, x))
+    print("decode T=2 (fused kernel, several tokens)", _forward_check(layer, ol, x[:2]))
+    print("decode T=4 (fused kernel, several tokens)", _forward_check(layer, ol, x[:4]))
+    print("decode T=5 (fused kernel, several tokens)", _forward_check(layer, ol, x[:5]))
+    print("decode T=8 (fused kernel, several tokens)", _forward_check(layer, ol, x[:8]))
+    print("decode T=9 (GEMV chain)", _forward_check(layer, ol, x[:9]))
+    print("decode T=16 (GEMV chain)", _forward_check(layer, ol, x))
     # the same tokens through the prefill path agree too
     layer2 = _layer(w, shape, max_tokens=4096, decode_max_tokens=0)
     print("prefill T=16", _forward_check(layer2, ol, x))
