@@ -71,9 +71,8 @@ extern "C" {
 
 /* ---- configuration flags ---------------------------------------------------------------------- */
 #define MOE_FLAG_ROUTER_SIMT     0x1u  /* compute the router on CUDA cores for every T */
-#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* decode calls of T <= 8 tokens: use the multi-kernel
-                                          GEMV chain instead of the fused decode kernel (one
-                                          launch for all the call's tokens, up to 8) */
+#define MOE_FLAG_DECODE_UNFUSED  0x2u  /* decode calls: use the multi-kernel GEMV chain instead
+                                          of the fused decode kernel (one launch per 8 tokens) */
 #define MOE_FLAG_POISON_WORKSPACE 0x4u /* test aid: the handle's workspace starts filled with 0xFF
                                           bytes (NaN floats, -1 indices) instead of zeros, except
                                           the words the kernels count on starting at zero, so a

@@ -211,8 +211,13 @@ def test_full_decode_workload(layer_idx):
     print("decode T=4 (fused kernel, several tokens)", _forward_check(layer, ol, x[:4]))
     print("decode T=5 (fused kernel, several tokens)", _forward_check(layer, ol, x[:5]))
     print("decode T=8 (fused kernel, several tokens)", _forward_check(layer, ol, x[:8]))
-    print("decode T=9 (GEMV chain)", _forward_check(layer, ol, x[:9]))
-    print("decode T=16 (GEMV chain)", _forward_check(layer, ol, x))
+    print("decode T=9 (fused kernel, 8 + 1 tokens)", _forward_check(layer, ol, x[:9]))
+    print("decode T=16 (fused kernel, 8 + 8 tokens)", _forward_check(layer, ol, x))
+    # the multi-kernel GEMV chain, which serves shapes the fused kernel does not fit
+    chain = _layer(w, shape, max_tokens=4096, decode_max_tokens=16, flags=M.MOE_FLAG_DECODE_UNFUSED)
+    for T in (1, 2, 9, 16):
+        print(f"decode T={T} (GEMV chain)", _forward_check(chain, ol, x[:T]))
+    chain.close()
     # the same tokens through the prefill path agree too
     layer2 = _layer(w, shape, max_tokens=4096, decode_max_tokens=0)
     print("prefill T=16", _forward_check(layer2, ol, x))
