@@ -510,6 +510,49 @@ def run_configs(args, dist, peaks, peak_src):
     return out
 
 
+def run_ep_single(args):
+    """The expert-parallel layer (bit_grouped_expert_router_b200.ep) with one rank, beside
+    moe_forward on the same layer and 4096-token chunk: eager calls, CUDA events around whole
+    forward calls (the EP forward reads its all-to-all split sizes back to the host once per call)."""
+    import torch
+    from bit_grouped_expert_router_b200 import _lib as M
+    from bit_grouped_expert_router_b200 import synth
+    from bit_grouped_expert_router_b200.ep import Exchange, ExpertParallelLayer, LibraryShard
+    shape = synth.WORKLOADS["prefill16k_zipf"]
+    w = synth.make_layer(shape, 0, device="cuda")
+    x = synth.make_x(shape, 0, 0, device="cuda")
+    full = M.Layer.from_shape(w, shape, max_tokens=shape.T, decode_max_tokens=16)
+    shard = LibraryShard(w, shape.H, shape.I, shape.E, shape.k, shape.has_shared, 0, 1, max_tokens=shape.T)
+    ep = ExpertParallelLayer(shard, Exchange(None, 1))
+    del w
+
+    def time_us(fn, reps=max(args.steps, 5)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1000.0 / reps
+
+    out = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, device="cuda")
+    t_full = time_us(lambda: full.forward(x, out=out))
+    t_ep = time_us(lambda: ep.forward(x))
+    diff = (ep.forward(x).float() - full.forward(x).float()).abs().max().item()
+    assert full.status() == 0
+    for L in (shard.router, shard.experts, shard.shared):
+        assert L.status() == 0
+    full.close()
+    shard.close()
+    return {"ranks": 1, "tokens": shape.T, "moe_forward_us": round(t_full, 1), "ep_forward_us": round(t_ep, 1),
+            "max_abs_diff_vs_moe_forward": round(diff, 4),
+            "note": "one rank: route, dispatch plan, row gather, routing-supplied expert forward, shared "
+                    "expert, combine; the all-to-all is a local copy"}
+
+
 def run_ablations(args, dist):
     """The pages' prefill levers, each against the product path on the same 4 layers (eager calls,
     CUDA events): GPU-resident routing vs a host round trip between routing and the expert GEMMs
@@ -762,6 +805,11 @@ def main():
             line["other_configs"] = run_configs(args, dist, peaks, peak_src)
         if args.ablations and dist.world == 1:
             line["ablations"] = run_ablations(args, dist)
+        if not args.no_configs and dist.world == 1:
+            try:   # a measurement beside the line: must never cost the line itself
+                line["expert_parallel"] = run_ep_single(args)
+            except Exception as e:   # noqa: BLE001
+                line["expert_parallel"] = {"error": f"{type(e).__name__}: {e}"[:300]}
         line["config"] = prefill_config(args, shape, r["n_layers"])
     base = {"n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16", "data": "synthetic (seeded random-init weights and activations)"}
