@@ -736,11 +736,17 @@ polled:
     __syncthreads();
     if (ok) {
         for (int t = 0; t < T; ++t) {
-            for (int i = tid; i < g.DM * 128; i += kDThreads) {
-                if (!s.ints[kIntFlags + t * kMaxDM + (i >> 7)]) continue;
-                const size_t hrow = (size_t)g.DM * r * 128 + i;
-                const float v = atomicExch(c.dfz.outacc + (size_t)t * H + hrow, 0.f);
-                c.out[(size_t)t * H + hrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            // four rows per thread: 16-byte reads at L2 (after the counter's acquire, through the
+            // barrier) and zeroing stores, 8-byte bf16 stores
+            for (int i4 = tid; 4 * i4 < g.DM * 128; i4 += kDThreads) {
+                if (!s.ints[kIntFlags + t * kMaxDM + ((4 * i4) >> 7)]) continue;
+                const size_t hrow = (size_t)g.DM * r * 128 + 4 * (size_t)i4;
+                float4* src = reinterpret_cast<float4*>(c.dfz.outacc + (size_t)t * H + hrow);
+                const float4 v = __ldcg(src);
+                __stcg(src, make_float4(0.f, 0.f, 0.f, 0.f));
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+                *reinterpret_cast<uint2*>(c.out + (size_t)t * H + hrow) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
             }
             if (tid < g.DM && s.ints[kIntFlags + t * kMaxDM + tid])
                 atomicExch(c.dfz.cnt + (size_t)t * MTd + g.DM * (int)r + tid, 0u);
