@@ -108,7 +108,9 @@ struct GemmCfg {
     static_assert(kSmemBytes * CTAS <= 227 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g * u / (1.f + __expf(-g)); }
+// silu(g) * u with the fast divide (a reciprocal and a multiply, within 2 ulp; the result is
+// rounded to fp16 next); a denominator past 2^126 (g < -87) gives 0, the limit of silu there
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.f + __expf(-g)); }
 
 __device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c, int bn) {
     return t.x >= 0 && t.x < c.G && t.y >= 0 && t.z > 0 && t.z <= bn && t.y + t.z <= c.rows_cap;
