@@ -392,9 +392,11 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             if (GATEUP) {
                 const int ilocal = 16 * q + (lane & 15);
                 const bool is_gate = lane < 16;
+                float amax = 0.f;   // largest |act| of this lane's valid columns (fp16 range check)
                 for (int c0 = 32 * eh; c0 < nvalid; c0 += 32 * (kEpiWarps / 4)) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
+                    const int lim = nvalid - c0 - (is_gate ? 0 : 16);   // this lane's valid r: r < lim
 #pragma unroll
                     for (int r = 0; r < 16; ++r) {
                         const float mine_lo = __uint_as_float(v[r]);
@@ -404,10 +406,12 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                         const float U = is_gate ? recv : mine_hi;
                         const int col = c0 + r + (is_gate ? 0 : 16);
                         const float a = silu_mul(G, U);
-                        if (col < nvalid && !(fabsf(a) <= 65504.f)) range_bad = true;
+                        if (lim >= 16 || r < lim) amax = fmaxf(amax, fabsf(a));
                         stage[col * 64 + ilocal] = __float2half_rn(a);  // columns >= nvalid: not copied out
                     }
                 }
+                // (a NaN activation can only come from a NaN x, which the fp16 copy of x reports)
+                if (!(amax <= 65504.f)) range_bad = true;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&accempty[ab]);
