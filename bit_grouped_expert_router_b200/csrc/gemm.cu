@@ -36,16 +36,17 @@
 //                    instructions of one scalar red per element, which made the down GEMM ~30 %
 //                    faster on this part (the scalar form was bound by the epilogue's issue).
 //
-// Warp roles (one persistent CTA per SM with 576 threads and 256-token tiles, or two per SM with
-// 320 threads and 128-token tiles -- GemmCfg; tiles taken round-robin from the device-built tile
+// Warp roles (one persistent CTA per SM with 640 threads and 256-token tiles, or two per SM with
+// 352 threads and 128-token tiles -- GemmCfg; tiles taken round-robin from the device-built tile
 // list so no tile count ever travels to the host):
-//   warp 0      TMA producer (lane 0)
+//   warp 0      token-tile TMA producer (lane 0)
 //   warp 1      TMEM allocator + MMA issuer (one lane)
-//   transform   warps 2-9 (or 2-5): dequantise a block into the A ring (thread = row, half of the
-//               64 columns; both halves with 4 warps)
-//   epilogue    warps 10-17 (or 6-9): drain a TMEM accumulator (double-buffered, so it overlaps
+//   epilogue    warps 2-9 (or 2-5): drain a TMEM accumulator (double-buffered, so it overlaps
 //               the next tile; warp w reads TMEM lanes 32*(w%4)..+31, the warps of a lane quarter
 //               take alternate 32-column chunks)
+//   transform   warps 10-12, 14-16, 18-19 (or 6-8, 10): dequantise a block into the A ring
+//               (thread = row, half of the 64 columns; both halves with 4 warps)
+//   warp 13 (or 9)  weight-block producer (lane 0); warp 17 idles
 // TMEM: two fp32 accumulators of kBN columns.  Every wait is bounded (common.cuh); on a timeout the
 // roles unwind, the producer waits for its copies in flight, the MMA thread waits for its MMAs,
 // and warp 1 frees the TMEM.
@@ -74,7 +75,8 @@ struct GemmCfg {
     // scheduler with the busy transform warps (measured: a tcgen05.mma issue took ~110 cycles
     // when it did, against ~45 alone), so the epilogue warps (idle between tiles) take warps
     // 2 .. 2 + kEpiWarps - 1 and the transform warps the following warps whose index is not 1
-    // mod 4; those left over stay idle.
+    // mod 4; the first of those left over issues the weight copies (a thread that mostly sleeps
+    // in mbarrier waits), the other stays idle.
     static constexpr int kEpiWarp0 = 2;
     static constexpr int kXWarp0 = 2 + kEpiWarps;   // first transform-candidate warp
     static constexpr int kXCand = kTransformWarps + (kTransformWarps - 1) / 3;   // skipping every 4th
@@ -197,9 +199,9 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         // Lane 0 waits for ring slots and issues the copies (the rest of the warp follows along).
         if (!(c.flags & 0x100u)) {
             const int shared_base = (GATEUP && c.has_shared) ? c.offsets[c.E] : 0;
-            uint32_t wit = 0, bit = 0, ait = 0;
-            int ws = 0, bs = 0, as = 0;
-            uint32_t wph = 0, bph = 0, aph = 0;
+            uint32_t bit = 0, ait = 0;
+            int bs = 0, as = 0;
+            uint32_t bph = 0, aph = 0;
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
                 const int mt = tau % MT;
@@ -210,7 +212,6 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 const CUtensorMap* map = &maps.m[from_x ? 1 : 0][hsel];
                 const int y = from_x ? tile.y - shared_base : tile.y;
                 const uint32_t b_bytes = (uint32_t)token_box_rows(hsel) * 128;
-                const uint8_t* wsrc = wbase + ((size_t)tile.x * MT + mt) * KS * kBlockBytes;
                 for (int kc = 0; kc < KS; ++kc) {
                     int ok = 1;
                     if (lane == 0 && AHBM) {   // the fp16 A tile of this k-step from HBM
@@ -223,18 +224,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                         }
                     }
                     if (lane == 0 && ok) {
-                        if (!AHBM && kc % kWB == 0) {
-                            const int nb = min(kWB, KS - kc);
-                            ok = mbar_wait(&wempty[ws], wph ^ 1u, abort_flag, c.status) ? 1 : 0;
-                            if (ok) {
-                                mbar_arrive_expect_tx(&wfull[ws], (uint32_t)nb * kBlockBytes);
-                                bulk_g2s(wsm + ws * kWStageBytes, wsrc + (size_t)kc * kBlockBytes,
-                                         (uint32_t)nb * kBlockBytes, &wfull[ws]);
-                                ++wit;
-                                if (++ws == kWS) { ws = 0; wph ^= 1u; }
-                            }
-                        }
-                        if (ok) ok = mbar_wait(&bempty[bs], bph ^ 1u, abort_flag, c.status) ? 1 : 0;
+                        ok = mbar_wait(&bempty[bs], bph ^ 1u, abort_flag, c.status) ? 1 : 0;
                         if (ok) {
                             mbar_arrive_expect_tx(&bfull[bs], b_bytes);
                             tma_load_2d(bsm + bs * kBTileBytes, map, kc * 64, y, &bfull[bs]);
@@ -249,8 +239,6 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         producer_done:
             // every copy issued must land before the CTA may exit
             if (lane == 0) {
-                for (uint32_t i = wit > (uint32_t)kWS ? wit - kWS : 0u; i < wit; ++i)
-                    mbar_drain(&wfull[i % kWS], (i / kWS) & 1u);
                 for (uint32_t i = bit > (uint32_t)kBS ? bit - kBS : 0u; i < bit; ++i)
                     mbar_drain(&bfull[i % kBS], (i / kBS) & 1u);
                 for (uint32_t i = ait > (uint32_t)kAS ? ait - kAS : 0u; i < ait; ++i)
@@ -300,6 +288,34 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 tc_commit(drainbar);
                 mbar_drain(drainbar, 0);
             }
+        }
+    } else if (warp == K::kXWarp0 + 3) {
+        // ------------------------------------------------------------------ weight producer
+        // Lane 0 refills each weight stage as soon as the transform warps release it, so the
+        // 4-bit blocks run up to kWS * kWB k-steps ahead of the transform whatever the token
+        // ring's state (sharing the token producer's thread tied their lead to the token ring's).
+        if (!AHBM && !(c.flags & 0x100u) && lane == 0) {
+            uint32_t wit = 0, wph = 0;
+            int ws = 0;
+            for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+                const int4 tile = c.tiles1[tau / MT];
+                const int mt = tau % MT;
+                if (!tile_ok(tile, c, kBN)) continue;
+                const uint8_t* wsrc = wbase + ((size_t)tile.x * MT + mt) * KS * kBlockBytes;
+                for (int kc = 0; kc < KS; kc += kWB) {
+                    const int nb = min(kWB, KS - kc);
+                    if (!mbar_wait(&wempty[ws], wph ^ 1u, abort_flag, c.status)) goto wproducer_done;
+                    mbar_arrive_expect_tx(&wfull[ws], (uint32_t)nb * kBlockBytes);
+                    bulk_g2s(wsm + ws * kWStageBytes, wsrc + (size_t)kc * kBlockBytes, (uint32_t)nb * kBlockBytes,
+                             &wfull[ws]);
+                    ++wit;
+                    if (++ws == kWS) { ws = 0; wph ^= 1u; }
+                }
+            }
+        wproducer_done:
+            // every copy issued must land before the CTA may exit
+            for (uint32_t i = wit > (uint32_t)kWS ? wit - kWS : 0u; i < wit; ++i)
+                mbar_drain(&wfull[i % kWS], (i / kWS) & 1u);
         }
     } else if (warp >= K::kXWarp0) {
         // ------------------------------------------------------------------ transform
