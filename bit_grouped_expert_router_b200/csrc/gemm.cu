@@ -14,12 +14,11 @@
 // Shaped by measurement on this part: every TMA operation costs an SM at least ~360 cycles
 // whatever its size, while big copies stream at ~90 B/clk.  So the weight blocks travel several
 // k-steps per copy, the token tile is a single box per k-step whose height (64/128/256 rows)
-// follows the tile's token count, and the three operand rings are sized separately (the token
-// ring's refill waits on L2, the A ring's only on the transform warps):
-//   weight ring  kWS stages x kWB blocks   (producer -> transform)
-//   token ring   kBS stages x kBN x 64     (producer -> MMA)
-//   A ring       kAS stages x 128 x 64     (transform -> MMA)
-// Barrier arrivals are one per warp.
+// follows the tile's token count, and the weight ring is sized apart from the operand stages:
+//   weight ring     kWS stages x kWB blocks               (weight producer -> transform)
+//   operand stages  kBS x (kBN x 64 tokens + 128 x 64 A)  (producer + transform -> MMA)
+// A stage's token tile and A tile share one full and one empty barrier, so the MMA-issuing thread
+// takes one wait and one commit per k-step.  Barrier arrivals are one per warp.
 //
 //   gate/up kernel : per tile (expert, 128 interleaved gate/up rows, <= kBN tokens), K = H.
 //                    B = the expert's bucketed fp16 token rows (the shared expert reads the fp16
@@ -85,8 +84,8 @@ struct GemmCfg {
     static constexpr int kAccCols = kBN;
     static constexpr int kWB = CTAS == 1 ? 4 : 2;   // weight blocks per bulk copy
     static constexpr int kWS = 2;                   // weight ring stages
-    static constexpr int kBS = CTAS == 1 ? 3 : 2;   // token ring stages
-    static constexpr int kAS = CTAS == 1 ? 3 : 2;   // A ring stages
+    static constexpr int kBS = CTAS == 1 ? 3 : 2;   // operand stages (one token tile + one A tile each)
+    static constexpr int kAS = kBS;
     static constexpr int kATileBytes = 128 * 128;   // 128 weight rows x 64 fp16
     static constexpr int kBTileBytes = kBN * 128;   // up to kBN token rows x 64 fp16
     static constexpr int kWStageBytes = kWB * kBlockBytes;
@@ -98,7 +97,7 @@ struct GemmCfg {
     static constexpr int kOffMeta = kOffStage + kStageBytes;
     static constexpr int kMetaBytes = 2 * kBN * 16; // [2 buffers][kBN] row pointer + gate (+ pad)
     static constexpr int kOffBar = kOffMeta + kMetaBytes;
-    static constexpr int kNumBars = 2 * (kWS + kBS + kAS) + 5;
+    static constexpr int kNumBars = 2 * (kWS + kBS) + 5;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kBN <= moe::kBN, "tile lists are sized for at most kBN rows per tile");
@@ -144,11 +143,13 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* wfull = bars;                 // weight blocks landed          (1 arrive + tx)
     uint64_t* wempty = wfull + kWS;         // weight blocks consumed        (1 arrive per transform warp)
-    uint64_t* bfull = wempty + kWS;         // token tile landed             (1 arrive + tx)
-    uint64_t* bempty = bfull + kBS;         // token tile's MMAs done        (commit)
-    uint64_t* afull = bempty + kBS;         // fp16 A tile written           (1 arrive per transform warp)
-    uint64_t* aempty = afull + kAS;         // A tile's MMAs done            (commit)
-    uint64_t* accfull = aempty + kAS;       // accumulator ready             (commit)
+    // One barrier pair per operand stage: the stage is full when its token tile has landed (the
+    // producer's arrive + tx) and its A tile is written (one arrive per transform warp, or the A
+    // tile's tx as well when A comes from HBM), and empty when its MMAs are done (one commit).
+    // The MMA thread thus takes one wait and one commit per k-step.
+    uint64_t* sfull = wempty + kWS;         // stage's token + A tiles ready (1 + transform arrives, + tx)
+    uint64_t* sempty = sfull + kBS;         // stage's MMAs done             (commit)
+    uint64_t* accfull = sempty + kBS;       // accumulator ready             (commit)
     uint64_t* accempty = accfull + 2;       // accumulator drained           (1 arrive per epilogue warp)
     uint64_t* drainbar = accfull + 4;       // MMA drain on abort            (commit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -165,12 +166,8 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             mbar_init(&wempty[s], kTransformWarps);
         }
         for (int s = 0; s < kBS; ++s) {
-            mbar_init(&bfull[s], 1);
-            mbar_init(&bempty[s], 1);
-        }
-        for (int s = 0; s < kAS; ++s) {
-            mbar_init(&afull[s], AHBM ? 1 : kTransformWarps);
-            mbar_init(&aempty[s], 1);
+            mbar_init(&sfull[s], AHBM ? 1 : 1 + kTransformWarps);
+            mbar_init(&sempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accfull[b], 1);
@@ -199,9 +196,9 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         // Lane 0 waits for ring slots and issues the copies (the rest of the warp follows along).
         if (!(c.flags & 0x100u)) {
             const int shared_base = (GATEUP && c.has_shared) ? c.offsets[c.E] : 0;
-            uint32_t bit = 0, ait = 0;
-            int bs = 0, as = 0;
-            uint32_t bph = 0, aph = 0;
+            uint32_t bit = 0;
+            int bs = 0;
+            uint32_t bph = 0;
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
                 const int4 tile = c.tiles1[tau / MT];
                 const int mt = tau % MT;
@@ -214,20 +211,13 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 const uint32_t b_bytes = (uint32_t)token_box_rows(hsel) * 128;
                 for (int kc = 0; kc < KS; ++kc) {
                     int ok = 1;
-                    if (lane == 0 && AHBM) {   // the fp16 A tile of this k-step from HBM
-                        ok = mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status) ? 1 : 0;
+                    if (lane == 0) {
+                        ok = mbar_wait(&sempty[bs], bph ^ 1u, abort_flag, c.status) ? 1 : 0;
                         if (ok) {
-                            mbar_arrive_expect_tx(&afull[as], (uint32_t)kATileBytes);
-                            tma_load_2d(asm_ + as * kATileBytes, &amap, kc * 64, (tile.x * MT + mt) * 128, &afull[as]);
-                            ++ait;
-                            if (++as == kAS) { as = 0; aph ^= 1u; }
-                        }
-                    }
-                    if (lane == 0 && ok) {
-                        ok = mbar_wait(&bempty[bs], bph ^ 1u, abort_flag, c.status) ? 1 : 0;
-                        if (ok) {
-                            mbar_arrive_expect_tx(&bfull[bs], b_bytes);
-                            tma_load_2d(bsm + bs * kBTileBytes, map, kc * 64, y, &bfull[bs]);
+                            mbar_arrive_expect_tx(&sfull[bs], b_bytes + (AHBM ? (uint32_t)kATileBytes : 0u));
+                            if (AHBM)   // the fp16 A tile of this k-step from HBM
+                                tma_load_2d(asm_ + bs * kATileBytes, &amap, kc * 64, (tile.x * MT + mt) * 128, &sfull[bs]);
+                            tma_load_2d(bsm + bs * kBTileBytes, map, kc * 64, y, &sfull[bs]);
                             ++bit;
                             if (++bs == kBS) { bs = 0; bph ^= 1u; }
                         }
@@ -237,20 +227,20 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 }
             }
         producer_done:
-            // every copy issued must land before the CTA may exit
+            // every copy issued must land before the CTA may exit (after an abort the transform
+            // warps may have left without their arrivals; the bounded drain then waits out its
+            // limit, far longer than any copy takes to land)
             if (lane == 0) {
                 for (uint32_t i = bit > (uint32_t)kBS ? bit - kBS : 0u; i < bit; ++i)
-                    mbar_drain(&bfull[i % kBS], (i / kBS) & 1u);
-                for (uint32_t i = ait > (uint32_t)kAS ? ait - kAS : 0u; i < ait; ++i)
-                    mbar_drain(&afull[i % kAS], (i / kAS) & 1u);
+                    mbar_drain(&sfull[i % kBS], (i / kBS) & 1u);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             uint32_t tl = 0;
-            int as = 0, bs = 0;
-            uint32_t aph = 0, bph = 0;
+            int bs = 0;
+            uint32_t bph = 0;
             bool issued = false;
             const uint32_t a0 = smem_u32(asm_), b0 = smem_u32(bsm);
             for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
@@ -265,19 +255,16 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 if (!mbar_wait(&accempty[ab], acph ^ 1u, abort_flag, c.status)) goto mma_done;
                 const uint32_t d_tmem = tmem + ab * kAccCols;
                 for (int kc = 0; kc < KS; ++kc) {
-                    if (!mbar_wait(&afull[as], aph, abort_flag, c.status)) goto mma_done;
-                    if (!mbar_wait(&bfull[bs], bph, abort_flag, c.status)) goto mma_done;
+                    if (!mbar_wait(&sfull[bs], bph, abort_flag, c.status)) goto mma_done;
                     tc_fence_after();
                     // descriptors of the stage once; the kk-th 16-column slice starts 32 bytes on,
                     // i.e. +2 in the start-address field (no carry: shared addresses < 256 KB)
-                    const uint64_t ad = sdesc_sw128(a0 + as * kATileBytes), bd = sdesc_sw128(b0 + bs * kBTileBytes);
+                    const uint64_t ad = sdesc_sw128(a0 + bs * kATileBytes), bd = sdesc_sw128(b0 + bs * kBTileBytes);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kc | kk) != 0 ? 1u : 0u);
                     issued = true;
-                    tc_commit(&aempty[as]);
-                    tc_commit(&bempty[bs]);
-                    if (++as == kAS) { as = 0; aph ^= 1u; }
+                    tc_commit(&sempty[bs]);
                     if (++bs == kBS) { bs = 0; bph ^= 1u; }
                 }
                 tc_commit(&accfull[ab]);
@@ -336,7 +323,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             for (int kc = 0; kc < KS; ++kc) {
                 // waits end the same way for the whole warp (the vote), so no lane is left behind
                 bool ok = kc % kWB != 0 || mbar_wait(&wfull[ws], wph, abort_flag, c.status);
-                ok = ok && mbar_wait(&aempty[as], aph ^ 1u, abort_flag, c.status);
+                ok = ok && mbar_wait(&sempty[as], aph ^ 1u, abort_flag, c.status);
                 if (!__all_sync(0xffffffffu, ok)) goto transform_done;
                 const uint8_t* blk = wsm + ws * kWStageBytes + (kc % kWB) * kBlockBytes;
 #pragma unroll
@@ -368,7 +355,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 }
                 fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[as]);
+                if (lane == 0) mbar_arrive(&sfull[as]);
                 if (++as == kAS) { as = 0; aph ^= 1u; }
                 if (kc % kWB == kWB - 1 || kc == KS - 1) {   // this weight stage is used up
                     if (lane == 0) mbar_arrive(&wempty[ws]);
