@@ -428,23 +428,39 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 named_bar(1, 32 * kEpiWarps);
             } else {
                 // tr[r][l] = accumulator (row 32q + l, token c0 + r); lane l then reads rows
-                // 32q + 4(l % 8) .. +3 of token c0 + 4g + l / 8 as one float4
+                // 32q + 4(l % 8) .. +3 of token c0 + 8(l / 8) + g as one float4, the gates and
+                // row pointers of its 8 consecutive tokens with 16-byte loads
                 float* tr = reinterpret_cast<float*>(stage) + (warp - kEpiWarp0) * 1024;
                 const int h4 = 32 * q + 4 * (lane & 7);   // first of this lane's 4 output rows
+                const int jl0 = 8 * (lane >> 3);          // first of this lane's 8 tokens of a chunk
                 for (int c0 = 32 * eh; c0 < nvalid; c0 += 32 * (kEpiWarps / 4)) {
                     uint32_t v[32];
                     tmem_ld32(taddr + c0, v);
 #pragma unroll
                     for (int r = 0; r < 32; ++r) tr[r * 32 + lane] = __uint_as_float(v[r]);
                     __syncwarp();
+                    float gts[8];
+                    float* rows[8];
+                    {
+                        const float4* gp = reinterpret_cast<const float4*>(meta_gate + ab * kBN + c0 + jl0);
+                        const float4 g0 = gp[0], g1 = gp[1];
+                        gts[0] = g0.x; gts[1] = g0.y; gts[2] = g0.z; gts[3] = g0.w;
+                        gts[4] = g1.x; gts[5] = g1.y; gts[6] = g1.z; gts[7] = g1.w;
+                        const ulonglong2* rp = reinterpret_cast<const ulonglong2*>(meta_row + ab * kBN + c0 + jl0);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const ulonglong2 pr = rp[u];
+                            rows[2 * u] = reinterpret_cast<float*>(pr.x);
+                            rows[2 * u + 1] = reinterpret_cast<float*>(pr.y);
+                        }
+                    }
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
-                        const int jl = 4 * g + (lane >> 3);
-                        const int j = c0 + jl;
-                        if (j < nvalid) {
+                        const int jl = jl0 + g;
+                        if (c0 + jl < nvalid) {
                             const float4 y = *reinterpret_cast<const float4*>(tr + jl * 32 + 4 * (lane & 7));
-                            const float gt = meta_gate[ab * kBN + j];
-                            red_add_v4(meta_row[ab * kBN + j] + h4, y.x * gt, y.y * gt, y.z * gt, y.w * gt);
+                            const float gt = gts[g];
+                            red_add_v4(rows[g] + h4, y.x * gt, y.y * gt, y.z * gt, y.w * gt);
                         }
                     }
                     __syncwarp();   // tr is rewritten by the next chunk
