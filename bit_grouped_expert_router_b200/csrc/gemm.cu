@@ -144,10 +144,11 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
     uint64_t* wfull = bars;                 // weight blocks landed          (1 arrive + tx)
     uint64_t* wempty = wfull + kWS;         // weight blocks consumed        (1 arrive per transform warp)
     // One barrier pair per operand stage: the stage is full when its token tile has landed (the
-    // producer's arrive + tx) and its A tile is written (one arrive per transform warp, or the A
+    // producer's arrive + tx) and its A tile is written (one arrive per warp of the transform group
+    // that took the k-step, or the A
     // tile's tx as well when A comes from HBM), and empty when its MMAs are done (one commit).
     // The MMA thread thus takes one wait and one commit per k-step.
-    uint64_t* sfull = wempty + kWS;         // stage's token + A tiles ready (1 + transform arrives, + tx)
+    uint64_t* sfull = wempty + kWS;         // stage's token + A tiles ready (1 + 4 transform arrives, + tx)
     uint64_t* sempty = sfull + kBS;         // stage's MMAs done             (commit)
     uint64_t* accfull = sempty + kBS;       // accumulator ready             (commit)
     uint64_t* accempty = accfull + 2;       // accumulator drained           (1 arrive per epilogue warp)
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             mbar_init(&wempty[s], kTransformWarps);
         }
         for (int s = 0; s < kBS; ++s) {
-            mbar_init(&sfull[s], AHBM ? 1 : 1 + kTransformWarps);
+            mbar_init(&sfull[s], AHBM ? 1 : 1 + 4);   // the producer, the k-step's 4 transform warps
             mbar_init(&sempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -306,14 +307,18 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         }
     } else if (warp >= K::kXWarp0) {
         // ------------------------------------------------------------------ transform
-        // thread = (weight row, half of the 64 columns; both halves when there are 4 transform
-        // warps); the fp16 pairs of 16-byte chunk ch of row r go to r*128 + ((ch ^ (r & 7)) * 16),
-        // the 128-byte swizzle the MMA descriptor expects.
+        // Groups of 4 warps, thread = weight row (both 64-column halves); with two groups (the
+        // one-CTA shape) they take alternate k-steps, so each warp converts a whole A tile's rows
+        // every second k-step and its waits, proxy fence and arrival serve twice the weights (the
+        // same per-warp work as in the two-CTA shape, whose k-steps per SM ran ~1.5x faster).
+        // The fp16 pairs of 16-byte chunk ch of row r go to r*128 + ((ch ^ (r & 7)) * 16), the
+        // 128-byte swizzle the MMA descriptor expects.
         const int wx = warp - K::kXWarp0;      // candidates: every warp not on scheduler 1
         const int ti = wx - (wx >> 2);          // transform warp index (when wx % 4 != 3)
         const bool active = !AHBM && (wx & 3) != 3 && ti < kTransformWarps;
-        const int tt = ti * 32 + lane;          // 0 .. 32 * kTransformWarps - 1
-        const int row = tt & 127;
+        constexpr int kXG = kTransformWarps / 4;   // groups; k-steps dealt round-robin (KS is even)
+        const int grp = ti >> 2;
+        const int row = (ti & 3) * 32 + lane;
         const uint32_t sw = (uint32_t)(row & 7);
         int ws = 0, as = 0;
         uint32_t wph = 0, aph = 0;
@@ -321,44 +326,49 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             const int4 tile = c.tiles1[tau / MT];
             if (!tile_ok(tile, c, kBN)) continue;
             for (int kc = 0; kc < KS; ++kc) {
-                // waits end the same way for the whole warp (the vote), so no lane is left behind
-                bool ok = kc % kWB != 0 || mbar_wait(&wfull[ws], wph, abort_flag, c.status);
-                ok = ok && mbar_wait(&sempty[as], aph ^ 1u, abort_flag, c.status);
-                if (!__all_sync(0xffffffffu, ok)) goto transform_done;
-                const uint8_t* blk = wsm + ws * kWStageBytes + (kc % kWB) * kBlockBytes;
+                const int kw = kc % kWB;   // block of the weight stage
+                if (kc % kXG == grp) {
+                    // waits end the same way for the whole warp (the vote), so no lane is left
+                    // behind; the group's first k-step of a weight stage waits for the stage
+                    bool ok = kw >= kXG || mbar_wait(&wfull[ws], wph, abort_flag, c.status);
+                    ok = ok && mbar_wait(&sempty[as], aph ^ 1u, abort_flag, c.status);
+                    if (!__all_sync(0xffffffffu, ok)) goto transform_done;
+                    const uint8_t* blk = wsm + ws * kWStageBytes + kw * kBlockBytes;
+                    const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+                    const uint4 cwh[2] = {*reinterpret_cast<const uint4*>(blk + row * 16),
+                                          *reinterpret_cast<const uint4*>(blk + 2048 + row * 16)};
+                    const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)),
+                                               __ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+                    const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)),
+                                               __ushort_as_half((unsigned short)(sb >> 16)));
+                    // codes of nibble position 1 (bits 4-7 of each 16-bit half) are read in place
+                    // as 16 q, so their scale is s / 16 (exact in fp16 for |s| >= 2^-13)
+                    const __half2 s2_16 = __hmul2(s2, __half2(__float2half(0.0625f), __float2half(0.0625f)));
+                    uint8_t* arow = asm_ + as * kATileBytes + row * 128;
 #pragma unroll
-                for (int hi = 0; hi < 8 / kTransformWarps; ++hi) {
-                const int half = kTransformWarps == 8 ? (tt >> 7) : hi;
-                const uint4 cw = *reinterpret_cast<const uint4*>(blk + half * 2048 + row * 16);
-                const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
-                const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)),
-                                           __ushort_as_half((unsigned short)(sb & 0xFFFFu)));
-                const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)),
-                                           __ushort_as_half((unsigned short)(sb >> 16)));
-                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-                // codes of nibble position 1 (bits 4-7 of each 16-bit half) are read in place as
-                // 16 q, so their scale is s / 16 (exact in fp16 for |s| >= 2^-13)
-                const __half2 s2_16 = __hmul2(s2, __half2(__float2half(0.0625f), __float2half(0.0625f)));
-                uint8_t* arow = asm_ + as * kATileBytes + row * 128;
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t words[4] = {cwh[half].x, cwh[half].y, cwh[half].z, cwh[half].w};
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const uint32_t lo = words[w], hi = words[w] >> 8;   // positions 0,1 | 2,3 (one shift)
-                    const __half2 v0 = __hfma2(nibble_pair_pos0(lo), s2, b2);
-                    const __half2 v1 = __hfma2(nibble_pair_pos1(lo), s2_16, b2);
-                    const __half2 v2 = __hfma2(nibble_pair_pos0(hi), s2, b2);
-                    const __half2 v3 = __hfma2(nibble_pair_pos1(hi), s2_16, b2);
-                    const uint32_t ch = (uint32_t)(4 * half + w);
-                    *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) =
-                        make_uint4(*reinterpret_cast<const uint32_t*>(&v0), *reinterpret_cast<const uint32_t*>(&v1),
-                                   *reinterpret_cast<const uint32_t*>(&v2), *reinterpret_cast<const uint32_t*>(&v3));
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t lo = words[w], hi = words[w] >> 8;   // positions 0,1 | 2,3 (one shift)
+                            const __half2 v0 = __hfma2(nibble_pair_pos0(lo), s2, b2);
+                            const __half2 v1 = __hfma2(nibble_pair_pos1(lo), s2_16, b2);
+                            const __half2 v2 = __hfma2(nibble_pair_pos0(hi), s2, b2);
+                            const __half2 v3 = __hfma2(nibble_pair_pos1(hi), s2_16, b2);
+                            const uint32_t ch = (uint32_t)(4 * half + w);
+                            *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(
+                                *reinterpret_cast<const uint32_t*>(&v0), *reinterpret_cast<const uint32_t*>(&v1),
+                                *reinterpret_cast<const uint32_t*>(&v2), *reinterpret_cast<const uint32_t*>(&v3));
+                        }
+                    }
+                    fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sfull[as]);
+                    // the group's last k-step of this weight stage releases it (one arrival per warp)
+                    if ((kw + kXG >= kWB || kc + kXG >= KS) && lane == 0) mbar_arrive(&wempty[ws]);
                 }
-                }
-                fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sfull[as]);
                 if (++as == kAS) { as = 0; aph ^= 1u; }
-                if (kc % kWB == kWB - 1 || kc == KS - 1) {   // this weight stage is used up
-                    if (lane == 0) mbar_arrive(&wempty[ws]);
+                if (kw == kWB - 1 || kc == KS - 1) {   // the stage's last k-step: every group moves on
                     if (++ws == kWS) { ws = 0; wph ^= 1u; }
                 }
             }
