@@ -317,6 +317,11 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         const int ti = wx - (wx >> 2);          // transform warp index (when wx % 4 != 3)
         const bool active = !AHBM && (wx & 3) != 3 && ti < kTransformWarps;
         constexpr int kXG = kTransformWarps / 4;   // groups; k-steps dealt round-robin (KS is even)
+        // A group's wait at k-step n (stage n % kAS, the MMAs of n - kAS done) is told apart from
+        // the stage's previous phase by parity only, so that phase (the MMAs of n - 2 kAS) must be
+        // complete when the group gets there: its wait at n - kXG guaranteed the MMAs of
+        // n - kXG - kAS, which covers it while kXG <= kAS.
+        static_assert(kXG <= kAS, "a transform group would reach a stage two phases ahead");
         const int grp = ti >> 2;
         const int row = (ti & 3) * 32 + lane;
         const uint32_t sw = (uint32_t)(row & 7);
