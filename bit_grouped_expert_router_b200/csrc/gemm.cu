@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
             mbar_init(&wempty[s], kTransformWarps);
         }
         for (int s = 0; s < kBS; ++s) {
-            mbar_init(&sfull[s], AHBM ? 1 : 1 + 4);   // the producer, the k-step's 4 transform warps
+            mbar_init(&sfull[s], AHBM ? 1 : 1 + (CTAS == 1 ? 4 : 2));   // the producer, the k-step's transform group
             mbar_init(&sempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -316,15 +316,16 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         const int wx = warp - K::kXWarp0;      // candidates: every warp not on scheduler 1
         const int ti = wx - (wx >> 2);          // transform warp index (when wx % 4 != 3)
         const bool active = !AHBM && (wx & 3) != 3 && ti < kTransformWarps;
-        constexpr int kXG = kTransformWarps / 4;   // groups; k-steps dealt round-robin (KS is even)
+        constexpr int kGW = CTAS == 1 ? 4 : 2;       // warps per group
+        constexpr int kRT = 4 / kGW;                 // weight rows per thread
+        constexpr int kXG = kTransformWarps / kGW;   // groups (2); k-steps dealt round-robin (KS is even)
         // A group's wait at k-step n (stage n % kAS, the MMAs of n - kAS done) is told apart from
         // the stage's previous phase by parity only, so that phase (the MMAs of n - 2 kAS) must be
         // complete when the group gets there: its wait at n - kXG guaranteed the MMAs of
         // n - kXG - kAS, which covers it while kXG <= kAS.
         static_assert(kXG <= kAS, "a transform group would reach a stage two phases ahead");
-        const int grp = ti >> 2;
-        const int row = (ti & 3) * 32 + lane;
-        const uint32_t sw = (uint32_t)(row & 7);
+        const int grp = ti / kGW;
+        const int row0 = (ti % kGW) * 32 + lane;   // rows row0, row0 + 128 / kRT, ...
         int ws = 0, as = 0;
         uint32_t wph = 0, aph = 0;
         for (int tau = active ? (int)blockIdx.x : total; tau < total; tau += gridDim.x) {
@@ -339,31 +340,36 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                     ok = ok && mbar_wait(&sempty[as], aph ^ 1u, abort_flag, c.status);
                     if (!__all_sync(0xffffffffu, ok)) goto transform_done;
                     const uint8_t* blk = wsm + ws * kWStageBytes + kw * kBlockBytes;
-                    const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
-                    const uint4 cwh[2] = {*reinterpret_cast<const uint4*>(blk + row * 16),
-                                          *reinterpret_cast<const uint4*>(blk + 2048 + row * 16)};
-                    const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)),
-                                               __ushort_as_half((unsigned short)(sb & 0xFFFFu)));
-                    const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)),
-                                               __ushort_as_half((unsigned short)(sb >> 16)));
-                    // codes of nibble position 1 (bits 4-7 of each 16-bit half) are read in place
-                    // as 16 q, so their scale is s / 16 (exact in fp16 for |s| >= 2^-13)
-                    const __half2 s2_16 = __hmul2(s2, __half2(__float2half(0.0625f), __float2half(0.0625f)));
-                    uint8_t* arow = asm_ + as * kATileBytes + row * 128;
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const uint32_t words[4] = {cwh[half].x, cwh[half].y, cwh[half].z, cwh[half].w};
+                    for (int rr = 0; rr < kRT; ++rr) {
+                        const int row = row0 + rr * (128 / kRT);
+                        const uint32_t sw = (uint32_t)(row & 7);
+                        const uint32_t sb = *reinterpret_cast<const uint32_t*>(blk + kBlockCodeBytes + row * 4);
+                        const uint4 cwh[2] = {*reinterpret_cast<const uint4*>(blk + row * 16),
+                                              *reinterpret_cast<const uint4*>(blk + 2048 + row * 16)};
+                        const __half2 s2 = __half2(__ushort_as_half((unsigned short)(sb & 0xFFFFu)),
+                                                   __ushort_as_half((unsigned short)(sb & 0xFFFFu)));
+                        const __half2 b2 = __half2(__ushort_as_half((unsigned short)(sb >> 16)),
+                                                   __ushort_as_half((unsigned short)(sb >> 16)));
+                        // codes of nibble position 1 (bits 4-7 of each 16-bit half) are read in
+                        // place as 16 q, so their scale is s / 16 (exact in fp16 for |s| >= 2^-13)
+                        const __half2 s2_16 = __hmul2(s2, __half2(__float2half(0.0625f), __float2half(0.0625f)));
+                        uint8_t* arow = asm_ + as * kATileBytes + row * 128;
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const uint32_t lo = words[w], hi = words[w] >> 8;   // positions 0,1 | 2,3 (one shift)
-                            const __half2 v0 = __hfma2(nibble_pair_pos0(lo), s2, b2);
-                            const __half2 v1 = __hfma2(nibble_pair_pos1(lo), s2_16, b2);
-                            const __half2 v2 = __hfma2(nibble_pair_pos0(hi), s2, b2);
-                            const __half2 v3 = __hfma2(nibble_pair_pos1(hi), s2_16, b2);
-                            const uint32_t ch = (uint32_t)(4 * half + w);
-                            *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(
-                                *reinterpret_cast<const uint32_t*>(&v0), *reinterpret_cast<const uint32_t*>(&v1),
-                                *reinterpret_cast<const uint32_t*>(&v2), *reinterpret_cast<const uint32_t*>(&v3));
+                        for (int half = 0; half < 2; ++half) {
+                            const uint32_t words[4] = {cwh[half].x, cwh[half].y, cwh[half].z, cwh[half].w};
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) {
+                                const uint32_t lo = words[w], hi = words[w] >> 8;   // positions 0,1 | 2,3 (one shift)
+                                const __half2 v0 = __hfma2(nibble_pair_pos0(lo), s2, b2);
+                                const __half2 v1 = __hfma2(nibble_pair_pos1(lo), s2_16, b2);
+                                const __half2 v2 = __hfma2(nibble_pair_pos0(hi), s2, b2);
+                                const __half2 v3 = __hfma2(nibble_pair_pos1(hi), s2_16, b2);
+                                const uint32_t ch = (uint32_t)(4 * half + w);
+                                *reinterpret_cast<uint4*>(arow + ((ch ^ sw) << 4)) = make_uint4(
+                                    *reinterpret_cast<const uint32_t*>(&v0), *reinterpret_cast<const uint32_t*>(&v1),
+                                    *reinterpret_cast<const uint32_t*>(&v2), *reinterpret_cast<const uint32_t*>(&v3));
+                            }
                         }
                     }
                     fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
