@@ -326,14 +326,18 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
         static_assert(kXG <= kAS, "a transform group would reach a stage two phases ahead");
         const int grp = ti / kGW;
         const int row0 = (ti % kGW) * 32 + lane;   // rows row0, row0 + 128 / kRT, ...
-        int ws = 0, as = 0;
-        uint32_t wph = 0, aph = 0;
+        // the group's k-steps only; ring positions from the k-steps of the CTA's earlier units (nb)
+        // (KS is a multiple of kWB, so weight stages start at unit boundaries)
+        uint32_t nb = 0;
         for (int tau = active ? (int)blockIdx.x : total; tau < total; tau += gridDim.x) {
             const int4 tile = c.tiles1[tau / MT];
             if (!tile_ok(tile, c, kBN)) continue;
-            for (int kc = 0; kc < KS; ++kc) {
+            for (int kc = grp; kc < KS; kc += kXG) {
                 const int kw = kc % kWB;   // block of the weight stage
-                if (kc % kXG == grp) {
+                const uint32_t n = nb + (uint32_t)kc, wchunk = n / kWB;
+                const int as = (int)(n % kAS), ws = (int)(wchunk % kWS);
+                const uint32_t aph = (n / kAS) & 1u, wph = (wchunk / kWS) & 1u;
+                {
                     // waits end the same way for the whole warp (the vote), so no lane is left
                     // behind; the group's first k-step of a weight stage waits for the stage
                     bool ok = kw >= kXG || mbar_wait(&wfull[ws], wph, abort_flag, c.status);
@@ -378,11 +382,8 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                     // the group's last k-step of this weight stage releases it (one arrival per warp)
                     if ((kw + kXG >= kWB || kc + kXG >= KS) && lane == 0) mbar_arrive(&wempty[ws]);
                 }
-                if (++as == kAS) { as = 0; aph ^= 1u; }
-                if (kw == kWB - 1 || kc == KS - 1) {   // the stage's last k-step: every group moves on
-                    if (++ws == kWS) { ws = 0; wph ^= 1u; }
-                }
             }
+            nb += (uint32_t)KS;
         }
     transform_done:;
     } else {
