@@ -80,7 +80,7 @@ struct Layout {
     size_t w_gu_bytes, w_dn_bytes, router_bytes, wsplit_bytes, weights_bytes;
     size_t o_wrt, o_rbias, o_sgw, o_router32;   // offsets inside the router region
     // workspace offsets
-    size_t o_part, o_idx, o_gates, o_sg, o_hist, o_counts, o_offsets, o_tiles, o_ntiles, o_perm, o_rtok,
+    size_t o_part, o_idx, o_gates, o_sg, o_hist, o_sdone, o_counts, o_offsets, o_tiles, o_ntiles, o_perm, o_rtok,
         o_rgate, o_x16, o_xp, o_act, o_acc, o_dact, o_dscale, o_status, o_stage_x, o_stage_out, o_dfz_ticket,
         o_dfz_slots, o_dfz_outacc, o_dfz_cnt, o_dfz_dirty, ws_bytes;
 };
@@ -131,6 +131,7 @@ Layout make_layout(const moe_config& c) {
     L.o_gates = take(sizeof(float) * (size_t)L.Tm * L.k);
     L.o_sg = take(sizeof(float) * (size_t)L.Tm);
     L.o_hist = take(sizeof(int) * (size_t)L.nblk_max * L.E);
+    L.o_sdone = take(sizeof(unsigned));
     L.o_counts = take(sizeof(int) * (size_t)(L.G + 1));
     L.o_offsets = take(sizeof(int) * (size_t)(L.G + 2));
     L.o_tiles = take(sizeof(int4) * (size_t)L.max_tiles);
@@ -322,8 +323,6 @@ int enqueue_routing(moe_handle* h, Prof& pf, const Ctx& c, bool decode, cudaStre
     MOE_LAUNCH("moe.topk", launch_topk(c, !decode, st));
     pf.mark(1);
     if (!decode) {
-        MOE_LAUNCH("moe.bucket_scan", launch_bucket_scan(c, st));
-        pf.mark(2);
         MOE_LAUNCH("moe.scatter", launch_scatter(c, st));
         pf.mark(3);
     }
@@ -440,11 +439,13 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     if (e != cudaSuccess) return cleanup(fail(MOE_ERR_CUDA, "cudaMalloc(workspace %zu B): %s", L.ws_bytes, cudaGetErrorString(e)));
     if (cfg->flags & MOE_FLAG_POISON_WORKSPACE) {
         // 0xFF bytes everywhere (NaN floats, -1 indices), then zero only the words the kernels
-        // count on starting at zero: the bucketing histograms, the status words and the fused
+        // count on starting at zero: the bucketing histograms and the scatter's finish counter,
+        // the status words and the fused
         // decode's call ticket and router words; its dirty word is raised, so the first decode
         // call resets its accumulator and counters on the device
         e = cudaMemsetAsync(h->ws, 0xFF, L.ws_bytes, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_hist, 0, sizeof(int) * (size_t)L.nblk_max * L.E, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_sdone, 0, sizeof(unsigned), st);
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_status, 0, sizeof(uint32_t) * 4, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(h->ws + L.o_dfz_ticket, 0, sizeof(unsigned long long), st);
         if (e == cudaSuccess)
@@ -525,6 +526,7 @@ int moe_create(const moe_config* cfg, const moe_weights* w, int device, void* st
     c.gates = reinterpret_cast<float*>(ws + L.o_gates);
     c.sg = reinterpret_cast<float*>(ws + L.o_sg);
     c.hist = reinterpret_cast<int*>(ws + L.o_hist);
+    c.scatter_done = reinterpret_cast<unsigned*>(ws + L.o_sdone);
     c.counts = reinterpret_cast<int*>(ws + L.o_counts);
     c.offsets = reinterpret_cast<int*>(ws + L.o_offsets);
     c.tiles1 = reinterpret_cast<int4*>(ws + L.o_tiles);
@@ -660,8 +662,6 @@ int moe_forward_routed(moe_handle* h, const uint16_t* x, int32_t T, const int32_
     MOE_LAUNCH("moe.routing_supplied", launch_routing_supplied(c, idx, gates, shared_gate, !decode, st));
     pf.mark(1);
     if (!decode) {
-        MOE_LAUNCH("moe.bucket_scan", launch_bucket_scan(c, st));
-        pf.mark(2);
         MOE_LAUNCH("moe.scatter", launch_scatter(c, st));
         pf.mark(3);
     }
@@ -713,7 +713,6 @@ int moe_route(moe_handle* h, const uint16_t* x, int32_t T, int32_t* idx, float* 
     if (rc != MOE_OK) return rc;
     if (decode) {
         MOE_LAUNCH("moe.topk", launch_topk(c, true, st));
-        MOE_LAUNCH("moe.bucket_scan", launch_bucket_scan(c, st));
         MOE_LAUNCH("moe.scatter", launch_scatter(c, st));
     }
     const Layout& L = h->L;

@@ -84,6 +84,7 @@ struct Ctx {
     float* gates;
     float* sg;
     int* hist;
+    unsigned* scatter_done;   // [1] scatter CTAs finished in this call (the last resets it to 0)
     int* counts;
     int* offsets;
     int4* tiles1;      // grouped-GEMM tile list {group, first bucket row, rows, 0}, ntiles[0] entries
@@ -116,7 +117,6 @@ int router_tc_splits();
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
 cudaError_t launch_routing_supplied(const Ctx& c, const int* idx, const float* gates, const float* sg,
                                     bool prefill, cudaStream_t st);
-cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st);
 
 // Rows of the token-tile TMA box with selector h: 64, 128 or 256 (a tile of n tokens loads the

@@ -5,14 +5,16 @@
 // This follows "Perplexity Open-Sources Lily..." section "The optimizations follow the
 // workload" (routing kept on the GPU, no CPU synchronisation during the MoE work).
 //
-// Bucketing is a stable counting sort done in three passes:
+// Bucketing is a stable counting sort done in two passes:
 //   topk      : per 64-token bucketing block, a histogram of its expert choices (global atomics);
-//   bucket_scan (one CTA): per-expert exclusive scan over the CTAs -> each CTA's base inside the
-//               bucket, bucket sizes, bucket offsets, and the tile list of the grouped GEMMs;
-//   scatter   : per CTA, ranks within the CTA in token order (warp match_any), giving every
-//               (token, slot) entry its row in the bucketed layout with its token and gate (the
-//               grouped GEMM gathers the token's activation row from there), and re-zeroes its
-//               histogram row for the next call.
+//   scatter   : every CTA (one per bucketing block) reads the whole histogram for the bucket sizes,
+//               the bucket offsets (exclusive scan over the experts) and its own base inside each
+//               bucket (the rows of earlier blocks); CTA 0 writes the sizes, offsets and the
+//               grouped GEMMs' tile list.  Then ranks within the CTA in token order (warp
+//               match_any) give every (token, slot) entry its row in the bucketed layout with its
+//               token and gate (the gather copies the token's activation row there), and the last
+//               CTA to finish re-zeroes the histogram for the next call.  (A separate one-CTA scan
+//               kernel between the two cost a kernel boundary on the critical path.)
 #include <float.h>
 
 #include "common.cuh"
@@ -283,7 +285,7 @@ cudaError_t launch_routing_supplied(const Ctx& c, const int* idx, const float* g
                       prefill ? 1 : 0);
 }
 
-// ---- bucket scan + tile list (one CTA) ---------------------------------------------------------
+// ---- bucket offsets + tile list, and the scatter ----------------------------------------------
 __device__ __forceinline__ int warp_incl_scan(int v) {
     const int lane = lane_id();
 #pragma unroll
@@ -294,47 +296,51 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
     return v;
 }
 
-// Four threads per expert each scan a quarter of the bucketing blocks (loads issued eight at a
-// time), the quarters are combined in shared memory, and a second pass writes every block's base
-// inside each bucket back into the histogram rows.
-__global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
+// ---- scatter: bucket positions and row metadata ---------------------------------------------
+
+__global__ void __launch_bounds__(1024) scatter_kernel(Ctx c) {
     griddep_wait();
     griddep_launch_dependents();
-    __shared__ int part[4][256];
-    __shared__ int cnt[264], off[264], toff[264];
-    const int tid = threadIdx.x, lane = lane_id();
-    const int e = tid & 255, quarter = tid >> 8;
-    const int b_lo = quarter * c.nblk / 4, b_hi = (quarter + 1) * c.nblk / 4;
-    int sum = 0;
-    if (e < c.E) {
-        for (int b0 = b_lo; b0 < b_hi; b0 += 8) {
-            int v[8];
+    __shared__ int part[4][256], partb[4][256];
+    __shared__ int cnt[264], off[264], toff[264];   // bucket sizes, offsets, first tile slots
+    __shared__ int last;
+    int* nxt = partb[0];    // [E] next free row of each bucket for this CTA (after the scan)
+    const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
+    const int b = blockIdx.x;
+    // Every CTA reads the whole histogram (one row per bucketing block): per expert the bucket
+    // size and this block's base inside the bucket (the rows of earlier blocks), four threads per
+    // expert each over a quarter of the blocks, loads issued eight at a time.  The L2 reads grow
+    // with the square of the blocks: 4 MB for 4096 tokens, 64 MB for 16384, 1 GB for 65536 (a
+    // few percent of a call that size).
+    {
+        const int e = tid & 255, quarter = tid >> 8;
+        const int b_lo = quarter * c.nblk / 4, b_hi = (quarter + 1) * c.nblk / 4;
+        int sum = 0, before = 0;
+        if (e < c.E) {
+            for (int b0 = b_lo; b0 < b_hi; b0 += 8) {
+                int v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = (b0 + u < b_hi) ? c.hist[(size_t)(b0 + u) * c.E + e] : 0;
+                for (int u = 0; u < 8; ++u) v[u] = (b0 + u < b_hi) ? c.hist[(size_t)(b0 + u) * c.E + e] : 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) sum += v[u];
-        }
-    }
-    part[quarter][e] = sum;
-    __syncthreads();
-    if (e < c.E) {
-        int run = 0;
-        for (int qq = 0; qq < quarter; ++qq) run += part[qq][e];
-        if (quarter == 3) cnt[e] = run + sum;
-        for (int b0 = b_lo; b0 < b_hi; b0 += 8) {
-            int v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = (b0 + u < b_hi) ? c.hist[(size_t)(b0 + u) * c.E + e] : 0;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (b0 + u < b_hi) c.hist[(size_t)(b0 + u) * c.E + e] = run;  // block base inside bucket e
-                run += v[u];
+                for (int u = 0; u < 8; ++u) {
+                    if (b0 + u < b) before += v[u];
+                    sum += v[u];
+                }
             }
         }
+        part[quarter][e] = sum;
+        partb[quarter][e] = before;
+    }
+    __syncthreads();
+    int mybase = 0;
+    if (tid < c.E) {
+        cnt[tid] = part[0][tid] + part[1][tid] + part[2][tid] + part[3][tid];
+        mybase = partb[0][tid] + partb[1][tid] + partb[2][tid] + partb[3][tid];
     }
     if (tid == 0 && c.has_shared) cnt[c.E] = c.T;
     __syncthreads();
-    if (tid < 32) {
+    // bucket offsets and the tile list's first slot of each group: exclusive scans in group order
+    if (warp == 0) {
         int run = 0, trun = 0;
         for (int base = 0; base < c.G; base += 32) {
             const int g = base + lane;
@@ -349,41 +355,26 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(Ctx c) {
         if (lane == 0) {
             off[c.G] = run;
             toff[c.G] = trun;
-            c.ntiles[0] = trun;
+            if (b == 0) c.ntiles[0] = trun;
         }
     }
     __syncthreads();
-    for (int g = tid; g <= c.G; g += blockDim.x) c.offsets[g] = off[g];
-    for (int g = tid; g < c.G; g += blockDim.x) c.counts[g] = cnt[g];
-    for (int g = tid; g < c.G; g += blockDim.x) {
-        const int n = cnt[g];
-        int tslot = toff[g];
-        for (int n0 = 0; n0 < n; n0 += c.tile_rows, ++tslot) {
-            if (tslot < c.max_tiles) c.tiles1[tslot] = make_int4(g, off[g] + n0, min(c.tile_rows, n - n0), 0);
-            else set_status(c.status, MOE_STATUS_BOUNDS);
+    if (tid < c.E) nxt[tid] = off[tid] + mybase;
+    if (b == 0) {   // the bucket sizes, offsets and tile list, once
+        for (int g = tid; g <= c.G; g += blockDim.x) c.offsets[g] = off[g];
+        for (int g = tid; g < c.G; g += blockDim.x) c.counts[g] = cnt[g];
+        for (int g = tid; g < c.G; g += blockDim.x) {
+            const int n = cnt[g];
+            int tslot = toff[g];
+            for (int n0 = 0; n0 < n; n0 += c.tile_rows, ++tslot) {
+                if (tslot < c.max_tiles) c.tiles1[tslot] = make_int4(g, off[g] + n0, min(c.tile_rows, n - n0), 0);
+                else set_status(c.status, MOE_STATUS_BOUNDS);
+            }
         }
     }
-}
-
-cudaError_t launch_bucket_scan(const Ctx& c, cudaStream_t st) {
-    return launch_pdl(bucket_scan_kernel, dim3(1), dim3(1024), 0, st, c);
-}
-
-// ---- scatter: bucket positions and row metadata ---------------------------------------------
-
-__global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
-    griddep_wait();
-    griddep_launch_dependents();
-    extern __shared__ int sm[];
-    int* cnt = sm;          // [E] next free row of each bucket for this CTA
-    const int lane = lane_id(), warp = threadIdx.x >> 5;
-    const int t0 = blockIdx.x * kTokPerBucketBlk;
+    __syncthreads();
+    const int t0 = b * kTokPerBucketBlk;
     const int nt = min(kTokPerBucketBlk, c.T - t0);
-    for (int e = threadIdx.x; e < c.E; e += blockDim.x) {
-        cnt[e] = c.offsets[e] + c.hist[(size_t)blockIdx.x * c.E + e];
-        c.hist[(size_t)blockIdx.x * c.E + e] = 0;   // ready for the next call's counting
-    }
-    __syncthreads();
     if (warp == 0) {
         // entries in (token, slot) order, 32 per step so equal experts keep that order (stable);
         // the expert ids and gates of 16 steps are loaded before those steps run
@@ -407,9 +398,9 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
                 if (active && (e < 0 || e >= c.E)) { set_status(c.status, MOE_STATUS_BOUNDS); e = 0; }
                 const unsigned mask = __match_any_sync(0xffffffffu, e);
                 const int rank = __popc(mask & ((1u << lane) - 1u));
-                const int p = active ? cnt[e] + rank : 0;
+                const int p = active ? nxt[e] + rank : 0;
                 __syncwarp();
-                if (active && lane == __ffs(mask) - 1) cnt[e] += __popc(mask);
+                if (active && lane == __ffs(mask) - 1) nxt[e] += __popc(mask);
                 __syncwarp();
                 if (active) {
                     if (p < 0 || p >= c.rows_cap) {
@@ -424,7 +415,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
         }
     }
     __syncthreads();
-    const int shared_base = c.offsets[c.E];
+    const int shared_base = off[c.E];
     if (c.has_shared) {
         for (int tt = threadIdx.x; tt < nt; tt += blockDim.x) {
             const int t = t0 + tt;
@@ -432,11 +423,22 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ctx c) {
             c.row_gate[shared_base + t] = c.sg[t];
         }
     }
+    // the last CTA to finish re-zeroes the histogram for the next call's counting (every CTA has
+    // read all of it by then) and resets the counter
+    if (tid == 0) {
+        __threadfence();
+        last = atomicAdd(c.scatter_done, 1u) == gridDim.x - 1 ? 1 : 0;
+    }
+    __syncthreads();
+    if (last) {
+        __threadfence();
+        for (int i = tid; i < c.nblk * c.E; i += blockDim.x) c.hist[i] = 0;
+        if (tid == 0) *c.scatter_done = 0u;
+    }
 }
 
 cudaError_t launch_scatter(const Ctx& c, cudaStream_t st) {
-    const size_t smem = sizeof(int) * (size_t)c.E;
-    return launch_pdl(scatter_kernel, dim3(c.nblk), dim3(256), smem, st, c);
+    return launch_pdl(scatter_kernel, dim3(c.nblk), dim3(1024), 0, st, c);
 }
 
 }  // namespace moe
