@@ -64,11 +64,15 @@ namespace {
 // MMA-issuing thread's chain of waits, issues and commits bounds a k-step at ~1000 cycles whatever
 // the tile's token count, so when experts get few tokens (tiles far from full) two independent
 // chains per SM win; when tiles are full, the larger tile's fewer k-steps win (host picks per call).
-template <int CTAS>
+template <int CTAS, bool GATEUP = true>
 struct GemmCfg {
     static_assert(CTAS == 1 || CTAS == 2, "CTAs per SM");
     static constexpr int kBN = CTAS == 1 ? 256 : 128;   // token columns per tile (= UMMA N)
-    static constexpr int kEpiWarps = 8 / CTAS;
+    // The one-CTA down GEMM takes 3 epilogue warps per TMEM lane quarter: its combine epilogue
+    // (transpose + vector reductions) of a full 256-token tile outlasts a unit's MMAs with 2, and
+    // the MMA thread then waits for the accumulator.
+    static constexpr int kEpiWarps = (CTAS == 1 && !GATEUP) ? 12 : 8 / CTAS;
+    static constexpr int kDnChunk = kEpiWarps > 8 ? 16 : 32;   // down epilogue: tokens per chunk
     static constexpr int kTransformWarps = 8 / CTAS;
     // Warp roles, placed by scheduler (warp % 4): the MMA-issuing warp 1 must not share its
     // scheduler with the busy transform warps (measured: a tcgen05.mma issue took ~110 cycles
@@ -102,7 +106,7 @@ struct GemmCfg {
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kBN <= moe::kBN, "tile lists are sized for at most kBN rows per tile");
     static_assert(2 * kAccCols <= kTmemCols, "TMEM budget");
-    static_assert(kStageBytes >= kEpiWarps * 32 * 32 * 4, "down epilogue: one 32 x 32 fp32 block per warp");
+    static_assert(kStageBytes >= kEpiWarps * kDnChunk * 32 * 4, "down epilogue: one chunk x 32 fp32 block per warp");
     static_assert(kOffB % 1024 == 0 && kOffW % 16 == 0 && kOffStage % 16 == 0 && kOffMeta % 16 == 0 &&
                       kOffBar % 8 == 0,
                   "align");
@@ -113,6 +117,22 @@ struct GemmCfg {
 // rounded to fp16 next); a denominator past 2^126 (g < -87) gives 0, the limit of silu there
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.f + __expf(-g)); }
 
+// tcgen05.ld, shape 32x32b, 16 columns: thread i of the warp reads TMEM lane (warp's quarter base +
+// i), registers r[j] = columns col..col+15 (the wait names the registers so no use moves above it).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c, int bn) {
     return t.x >= 0 && t.x < c.G && t.y >= 0 && t.z > 0 && t.z <= bn && t.y + t.z <= c.rows_cap;
 }
@@ -121,11 +141,11 @@ __device__ __forceinline__ bool tile_ok(const int4& t, const Ctx& c, int bn) {
 // tile per k-step, box 64 columns x 128 rows, the same 128-byte swizzle the transform writes)
 // instead of rebuilding it from the 4-bit blocks in shared memory; the transform warps idle.
 template <bool GATEUP, int CTAS, bool AHBM>
-__global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
+__global__ void __launch_bounds__(GemmCfg<CTAS, GATEUP>::kThreads, CTAS)
     grouped_gemm_kernel(Ctx c, const __grid_constant__ TokenMaps maps, const __grid_constant__ CUtensorMap amap) {
     griddep_wait();
     griddep_launch_dependents();
-    using K = GemmCfg<CTAS>;
+    using K = GemmCfg<CTAS, GATEUP>;
     constexpr int kBN = K::kBN, kEpiWarps = K::kEpiWarps, kTransformWarps = K::kTransformWarps;
     constexpr int kEpiWarp0 = K::kEpiWarp0, kTmemCols = K::kTmemCols, kAccCols = K::kAccCols;
     constexpr int kWB = K::kWB, kWS = K::kWS, kBS = K::kBS, kAS = K::kAS;
@@ -449,35 +469,40 @@ __global__ void __launch_bounds__(GemmCfg<CTAS>::kThreads, CTAS)
                 }
                 named_bar(1, 32 * kEpiWarps);
             } else {
-                // tr[r][l] = accumulator (row 32q + l, token c0 + r); lane l then reads rows
-                // 32q + 4(l % 8) .. +3 of token c0 + 8(l / 8) + g as one float4, the gates and
-                // row pointers of its 8 consecutive tokens with 16-byte loads
-                float* tr = reinterpret_cast<float*>(stage) + (warp - kEpiWarp0) * 1024;
+                // tr[r][l] = accumulator (row 32q + l, token c0 + r), kC tokens per chunk; lane l
+                // then reads rows 32q + 4(l % 8) .. +3 of token c0 + (kC / 4)(l / 8) + g as one
+                // float4, the gates and row pointers of its kC / 4 consecutive tokens with 16-byte
+                // loads
+                constexpr int kC = K::kDnChunk, kG = kC / 4;
+                float* tr = reinterpret_cast<float*>(stage) + (warp - kEpiWarp0) * (kC * 32);
                 const int h4 = 32 * q + 4 * (lane & 7);   // first of this lane's 4 output rows
-                const int jl0 = 8 * (lane >> 3);          // first of this lane's 8 tokens of a chunk
-                for (int c0 = 32 * eh; c0 < nvalid; c0 += 32 * (kEpiWarps / 4)) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + c0, v);
+                const int jl0 = kG * (lane >> 3);         // first of this lane's kG tokens of a chunk
+                for (int c0 = kC * eh; c0 < nvalid; c0 += kC * (kEpiWarps / 4)) {
+                    uint32_t v[kC];
+                    if constexpr (kC == 32) tmem_ld32(taddr + c0, v);
+                    else tmem_ld16(taddr + c0, v);
 #pragma unroll
-                    for (int r = 0; r < 32; ++r) tr[r * 32 + lane] = __uint_as_float(v[r]);
+                    for (int r = 0; r < kC; ++r) tr[r * 32 + lane] = __uint_as_float(v[r]);
                     __syncwarp();
-                    float gts[8];
-                    float* rows[8];
+                    float gts[kG];
+                    float* rows[kG];
                     {
                         const float4* gp = reinterpret_cast<const float4*>(meta_gate + ab * kBN + c0 + jl0);
-                        const float4 g0 = gp[0], g1 = gp[1];
-                        gts[0] = g0.x; gts[1] = g0.y; gts[2] = g0.z; gts[3] = g0.w;
-                        gts[4] = g1.x; gts[5] = g1.y; gts[6] = g1.z; gts[7] = g1.w;
+#pragma unroll
+                        for (int u = 0; u < kG / 4; ++u) {
+                            const float4 gq = gp[u];
+                            gts[4 * u] = gq.x; gts[4 * u + 1] = gq.y; gts[4 * u + 2] = gq.z; gts[4 * u + 3] = gq.w;
+                        }
                         const ulonglong2* rp = reinterpret_cast<const ulonglong2*>(meta_row + ab * kBN + c0 + jl0);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < kG / 2; ++u) {
                             const ulonglong2 pr = rp[u];
                             rows[2 * u] = reinterpret_cast<float*>(pr.x);
                             rows[2 * u + 1] = reinterpret_cast<float*>(pr.y);
                         }
                     }
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
+                    for (int g = 0; g < kG; ++g) {
                         const int jl = jl0 + g;
                         if (c0 + jl < nvalid) {
                             const float4 y = *reinterpret_cast<const float4*>(tr + jl * 32 + 4 * (lane & 7));
@@ -541,7 +566,7 @@ namespace {
 
 template <bool GATEUP, int CTAS, bool AHBM>
 cudaError_t launch_grouped(const Ctx& c, const TokenMaps& maps, const CUtensorMap& amap, int num_sms, cudaStream_t st) {
-    using K = GemmCfg<CTAS>;
+    using K = GemmCfg<CTAS, GATEUP>;
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, CTAS, AHBM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmemBytes);
     if (e != cudaSuccess) return e;
