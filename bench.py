@@ -301,7 +301,7 @@ def run_prefill(args, dist, peaks, peak_src):
               "us_per_chunk": round(t * 1e6, 1)}
         gg.update(tile_stats(layers, xs, shape, prof, clk))
     res = dict(value=value, ms=ms, clocks=clk, roofline=roof, kernels=prof, grouped_gemm=gg,
-               launches=8 * chunks * n_layers * args.steps, shape=shape, n_layers=n_layers,
+               launches=len(prof) * chunks * n_layers * args.steps, shape=shape, n_layers=n_layers,
                tokens_per_step=tokens_per_step)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
