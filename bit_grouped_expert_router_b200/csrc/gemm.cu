@@ -35,17 +35,19 @@
 //                    instructions of one scalar red per element, which made the down GEMM ~30 %
 //                    faster on this part (the scalar form was bound by the epilogue's issue).
 //
-// Warp roles (one persistent CTA per SM with 640 threads and 256-token tiles, or two per SM with
-// 352 threads and 128-token tiles -- GemmCfg; tiles taken round-robin from the device-built tile
-// list so no tile count ever travels to the host):
+// Warp roles (GemmCfg; tiles taken round-robin from the device-built tile list so no tile count
+// ever travels to the host).  kE epilogue warps: 4 for gate/up and the two-CTA shape, 16 for the
+// one-CTA down GEMM.
 //   warp 0      token-tile TMA producer (lane 0)
 //   warp 1      TMEM allocator + MMA issuer (one lane)
-//   epilogue    warps 2-9 (or 2-5): drain a TMEM accumulator (double-buffered, so it overlaps
-//               the next tile; warp w reads TMEM lanes 32*(w%4)..+31, the warps of a lane quarter
-//               take alternate 32-column chunks)
-//   transform   warps 10-12, 14-16, 18-19 (or 6-8, 10): dequantise a block into the A ring
-//               (thread = row, half of the 64 columns; both halves with 4 warps)
-//   warp 13 (or 9)  weight-block producer (lane 0); warp 17 idles
+//   epilogue    warps 2 .. 2+kE-1: drain a TMEM accumulator (double-buffered, so it overlaps the
+//               next tile; warp w reads TMEM lanes 32*(w%4)..+31, the warps of a lane quarter take
+//               alternate column chunks)
+//   transform   the next warps not on scheduler 1 (warp % 4 != 1), 8 (or 4 in the two-CTA shape),
+//               in groups taking alternate k-steps: dequantise a block into the A ring
+//   the first warp left on scheduler 1 issues the weight-block copies (lane 0); one more idles.
+// One CTA per SM: 512 threads for gate/up, 896 for down, 256-token tiles; two per SM: 352
+// threads, 128-token tiles.
 // TMEM: two fp32 accumulators of kBN columns.  Every wait is bounded (common.cuh); on a timeout the
 // roles unwind, the producer waits for its copies in flight, the MMA thread waits for its MMAs,
 // and warp 1 frees the TMEM.
@@ -71,8 +73,10 @@ struct GemmCfg {
     // The one-CTA down GEMM takes 4 epilogue warps per TMEM lane quarter: its combine epilogue
     // (transpose + vector reductions) of a full 256-token tile outlasts a unit's MMAs with 2, and
     // the MMA thread then waits for the accumulator (measured: 2 -> 3 -> 4 per quarter, down
-    // 139.3 -> 134.3 -> 130.8 us per 4096-token chunk; 5 would cap the registers at 64).
-    static constexpr int kEpiWarps = (CTAS == 1 && !GATEUP) ? 16 : 8 / CTAS;
+    // 139.3 -> 134.3 -> 130.8 us per 4096-token chunk; 5 would cap the registers at 64).  The
+    // gate/up epilogue (SwiGLU, ~1/3 of a unit's time with one warp per quarter) needs one; fewer
+    // warps beside the transform warps: gate/up 189.7 -> 188.6 us against two per quarter.
+    static constexpr int kEpiWarps = CTAS == 1 && !GATEUP ? 16 : 4;
     static constexpr int kDnChunk = kEpiWarps > 8 ? 16 : 32;   // down epilogue: tokens per chunk
     static constexpr int kTransformWarps = 8 / CTAS;
     // Warp roles, placed by scheduler (warp % 4): the MMA-issuing warp 1 must not share its
