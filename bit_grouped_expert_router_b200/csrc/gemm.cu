@@ -28,8 +28,8 @@
 //                    to the expert's act rows (only the tile's valid tokens).
 //   down kernel    : per tile (expert, 128 output rows, <= kBN tokens), K = I.  B = act rows.
 //                    Epilogue: y * gate (routing gate, or sigmoid gate for the shared expert) added
-//                    into the token's fp32 accumulator row.  A warp's 32 x 32 block (32 output
-//                    rows = TMEM lanes, 32 tokens) is transposed through shared memory so that each
+//                    into the token's fp32 accumulator row.  A warp's block (32 output rows = TMEM
+//                    lanes x 16 or 32 tokens) is transposed through shared memory so that each
 //                    lane adds 4 consecutive rows of one token with one red.global.add.v4.f32 (8
 //                    lanes cover a token's 128 contiguous bytes): a quarter of the reduction
 //                    instructions of one scalar red per element, which made the down GEMM ~30 %
@@ -60,12 +60,13 @@ namespace moe {
 
 namespace {
 
-// Two launch shapes of the same kernel.  CTAS = 1: one 576-thread CTA per SM, 256-token tiles,
-// rings of 3 token / 3 A stages and 4-block weight copies.  CTAS = 2: two 320-thread CTAs per SM
-// (half the roles and half the TMEM each), 128-token tiles, 2 + 2 stages and 2-block copies.  The
-// MMA-issuing thread's chain of waits, issues and commits bounds a k-step at ~1000 cycles whatever
-// the tile's token count, so when experts get few tokens (tiles far from full) two independent
-// chains per SM win; when tiles are full, the larger tile's fewer k-steps win (host picks per call).
+// Two launch shapes of the same kernel.  CTAS = 1: one CTA per SM (512 threads for gate/up, 896
+// for down), 256-token tiles, 3 operand stages and 4-block weight copies.  CTAS = 2: two 352-thread
+// CTAs per SM (half the roles and half the TMEM each), 128-token tiles, 2 stages and 2-block
+// copies.  A k-step costs about the same whatever the tile's token count (a ring of hand-offs
+// between the producers, the transform groups and the MMA-issuing thread), so when experts get
+// few tokens (tiles far from full) two independent rings per SM win; when tiles are full, the
+// larger tile's fewer k-steps win (host picks per call).
 template <int CTAS, bool GATEUP = true>
 struct GemmCfg {
     static_assert(CTAS == 1 || CTAS == 2, "CTAs per SM");
