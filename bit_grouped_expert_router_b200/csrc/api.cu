@@ -125,7 +125,8 @@ Layout make_layout(const moe_config& c) {
         o = align_up(o + bytes, 256);
         return at;
     };
-    const size_t part_rows = std::max((size_t)router_tc_splits() * L.Tm, (size_t)L.ks_dec * (size_t)L.Tdec);
+    size_t part_rows = (size_t)L.ks_dec * (size_t)L.Tdec;
+    for (int T = 1; T <= L.Tm; ++T) part_rows = std::max(part_rows, (size_t)router_tc_splits(T, L.H) * T);
     L.o_part = take(sizeof(float) * part_rows * L.E);
     L.o_idx = take(sizeof(int) * (size_t)L.Tm * L.k);
     L.o_gates = take(sizeof(float) * (size_t)L.Tm * L.k);
@@ -264,7 +265,7 @@ Ctx make_ctx(const moe_handle* h, int T, const uint16_t* x, uint16_t* out, bool 
     c.x = x;
     c.out = out;
     c.nblk = (T + kTokPerBucketBlk - 1) / kTokPerBucketBlk;
-    c.ks = decode ? h->L.ks_dec : ((h->cfg.flags & MOE_FLAG_ROUTER_SIMT) ? 1 : router_tc_splits());
+    c.ks = decode ? h->L.ks_dec : ((h->cfg.flags & MOE_FLAG_ROUTER_SIMT) ? 1 : router_tc_splits(T, h->L.H));
     return c;
 }
 

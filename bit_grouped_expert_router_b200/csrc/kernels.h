@@ -113,7 +113,7 @@ cudaError_t launch_router_split(const float* router, int H, int E, int Epad, uin
 cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmW, const CUtensorMap& tmX, int n_exp,
                              cudaStream_t st);
 int router_tc_smem_bytes();
-int router_tc_splits();
+int router_tc_splits(int T, int H);   // partial sums of the tensor-core router, T tokens of H
 cudaError_t launch_topk(const Ctx& c, bool histogram, cudaStream_t st);
 cudaError_t launch_routing_supplied(const Ctx& c, const int* idx, const float* gates, const float* sg,
                                     bool prefill, cudaStream_t st);

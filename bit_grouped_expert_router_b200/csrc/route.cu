@@ -185,6 +185,28 @@ __global__ void __launch_bounds__(256) topk_kernel(Ctx c, int do_hist) {
             const float s = (((pq[0][i] + pq[1][i]) + pq[2][i]) + pq[3][i]) + (e < c.E ? c.rbias[e] : 0.f);
             l[i] = (e < c.E && s == s) ? s : -INFINITY;
         }
+    } else if (c.ks % 4 == 0) {   // 8 or 16 partial sums (short calls): four splits' loads at a time
+        float sacc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sacc[i] = 0.f;
+        for (int q0 = 0; q0 < c.ks; q0 += 4) {
+            float pq[4][8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = lane + 32 * i;
+                    pq[q][i] = e < c.E ? c.part[((size_t)(q0 + q) * c.T + t) * c.E + e] : 0.f;
+                }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sacc[i] = (((sacc[i] + pq[0][i]) + pq[1][i]) + pq[2][i]) + pq[3][i];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            const float s = sacc[i] + (e < c.E ? c.rbias[e] : 0.f);
+            l[i] = (e < c.E && s == s) ? s : -INFINITY;
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {

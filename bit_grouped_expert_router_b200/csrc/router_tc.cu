@@ -4,8 +4,10 @@
 // two bf16 terms, W1 = bf16(W) and W2 = bf16(W - W1), which carry 16 significant bits of every
 // weight (relative residual <= 2^-17); x is bf16 already, so every product x*Wi is exact.  The
 // tensor core's fp32 accumulation does not round to nearest on every add, so long accumulation
-// chains drift: the K = 2H products of one logit are split four ways into separate partial sums
-// (each its own short chain on the tensor core) that the top-k kernel adds in fp32.  Measured
+// chains drift: the K = 2H products of one logit are split into 4 or more separate partial sums
+// (each its own short chain on the tensor core) that the top-k kernel adds in fp32, in split order.
+// Short calls take more splits (up to 16), so that their few token tiles still spread over the
+// SMs: 512 tokens are 4 tiles, 16 CTAs with four splits.  Measured
 // against the fp64 oracle the logits agree to a few 1e-6 -- far inside the 1e-3 top-(k+1) gap
 // the routing is checked with.  (The split-K SIMT router in route.cu serves decode-sized T.)
 //
@@ -22,7 +24,7 @@ namespace moe {
 namespace {
 
 constexpr int kRM = 128;        // tokens per CTA (UMMA M)
-constexpr int kRSplit = 4;      // K quarters (partial sums)
+constexpr int kRSplit = 4;      // K splits (partial sums) of calls with enough token tiles
 constexpr int kRStages = 4;
 constexpr int kRThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
 constexpr int kRAT = kRM * 128;  // bytes of the x tile
@@ -46,10 +48,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int t0 = blockIdx.x * kRM;
-    const int split = blockIdx.y;
+    const int split = blockIdx.y, nsplit = gridDim.y;
     const int KH = c.H / 64;                 // k-steps per term (the x tile repeats for each term)
     const int KS = 2 * KH;
-    const int k_begin = split * KS / kRSplit, k_end = (split + 1) * KS / kRSplit;
+    const int k_begin = split * KS / nsplit, k_end = (split + 1) * KS / nsplit;
     const int tmem_cols = n_exp <= 32 ? 32 : (n_exp <= 64 ? 64 : (n_exp <= 128 ? 128 : 256));
     const uint32_t b_bytes = (uint32_t)n_exp * 128;
 
@@ -122,6 +124,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
             for (int c0 = 0; c0 < n_exp; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + c0, v);
+                if (k_end <= k_begin) {   // a split without k-steps (never chosen): its sum is 0
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) v[r] = 0u;
+                }
                 if (t < c.T) {
                     if (c0 + 32 <= c.E && (c.E & 3) == 0) {
 #pragma unroll
@@ -164,7 +170,13 @@ __global__ void router_split_kernel(const float* __restrict__ router, int H, int
 }  // namespace
 
 int router_tc_smem_bytes() { return kRSmem; }
-int router_tc_splits() { return kRSplit; }
+int router_tc_splits(int T, int H) {
+    const int tiles = (T + kRM - 1) / kRM;
+    int s = kRSplit;
+    // at least two k-steps per split (2H / 64 k-steps in all); 148: the SMs of a B200
+    while (s < 16 && tiles * 2 * s <= 148 && 2 * s * 2 <= 2 * H / 64) s *= 2;
+    return s;
+}
 
 cudaError_t launch_router_split(const float* router, int H, int E, int Epad, uint16_t* wsplit, cudaStream_t st) {
     router_split_kernel<<<256, 256, 0, st>>>(router, H, E, Epad, wsplit);
@@ -176,7 +188,7 @@ cudaError_t launch_router_tc(const Ctx& c, const CUtensorMap& tmW, const CUtenso
                              cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
     if (e != cudaSuccess) return e;
-    dim3 grid((c.T + kRM - 1) / kRM, kRSplit);
+    dim3 grid((c.T + kRM - 1) / kRM, c.ks);
     return launch_pdl(router_tc_kernel, grid, dim3(kRThreads), kRSmem, st, c, n_exp, tmW, tmX);
 }
 
