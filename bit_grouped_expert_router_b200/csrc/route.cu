@@ -325,6 +325,8 @@ __global__ void __launch_bounds__(1024) scatter_kernel(Ctx c) {
     griddep_launch_dependents();
     __shared__ int part[4][256], partb[4][256];
     __shared__ int cnt[264], off[264], toff[264];   // bucket sizes, offsets, first tile slots
+    __shared__ int wtot[2][32];                     // per-warp totals of the group scan
+    __shared__ int wcnt[32 * 256];                  // [warp][expert] counts, then bases, of a round
     __shared__ int last;
     int* nxt = partb[0];    // [E] next free row of each bucket for this CTA (after the scan)
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
@@ -361,23 +363,29 @@ __global__ void __launch_bounds__(1024) scatter_kernel(Ctx c) {
     }
     if (tid == 0 && c.has_shared) cnt[c.E] = c.T;
     __syncthreads();
-    // bucket offsets and the tile list's first slot of each group: exclusive scans in group order
-    if (warp == 0) {
-        int run = 0, trun = 0;
-        for (int base = 0; base < c.G; base += 32) {
-            const int g = base + lane;
-            const int v = (g < c.G) ? cnt[g] : 0;
-            const int nt = (v + c.tile_rows - 1) / c.tile_rows;
-            const int inc = warp_incl_scan(v);
-            const int tinc = warp_incl_scan(nt);
-            if (g < c.G) { off[g] = run + inc - v; toff[g] = trun + tinc - nt; }
-            run += __shfl_sync(0xffffffffu, inc, 31);
-            trun += __shfl_sync(0xffffffffu, tinc, 31);
+    // bucket offsets and the tile list's first slot of each group: exclusive scans in group order,
+    // 32 groups per warp, then the warps' totals added in front
+    {
+        const int g = tid, nwg = (c.G + 31) / 32;
+        int v = 0, ntl = 0, inc = 0, tinc = 0;
+        if (warp < nwg) {
+            v = (g < c.G) ? cnt[g] : 0;
+            ntl = (v + c.tile_rows - 1) / c.tile_rows;
+            inc = warp_incl_scan(v);
+            tinc = warp_incl_scan(ntl);
+            if (lane == 31) { wtot[0][warp] = inc; wtot[1][warp] = tinc; }
         }
-        if (lane == 0) {
-            off[c.G] = run;
-            toff[c.G] = trun;
-            if (b == 0) c.ntiles[0] = trun;
+        __syncthreads();
+        if (warp < nwg && g < c.G) {
+            int pre = 0, tpre = 0;
+            for (int w = 0; w < warp; ++w) { pre += wtot[0][w]; tpre += wtot[1][w]; }
+            off[g] = pre + inc - v;
+            toff[g] = tpre + tinc - ntl;
+            if (g == c.G - 1) {
+                off[c.G] = pre + inc;
+                toff[c.G] = tpre + tinc;
+                if (b == 0) c.ntiles[0] = tpre + tinc;
+            }
         }
     }
     __syncthreads();
@@ -397,46 +405,53 @@ __global__ void __launch_bounds__(1024) scatter_kernel(Ctx c) {
     __syncthreads();
     const int t0 = b * kTokPerBucketBlk;
     const int nt = min(kTokPerBucketBlk, c.T - t0);
-    if (warp == 0) {
-        // entries in (token, slot) order, 32 per step so equal experts keep that order (stable);
-        // the expert ids and gates of 16 steps are loaded before those steps run
-        constexpr int kChunk = 16;
-        const int n_entries = nt * c.k;
-        for (int base0 = 0; base0 < n_entries; base0 += 32 * kChunk) {
-            int ev[kChunk];
-            float gv[kChunk];
-#pragma unroll
-            for (int u = 0; u < kChunk; ++u) {
-                const int i = base0 + 32 * u + lane;
-                ev[u] = i < n_entries ? c.idx[t0 * c.k + i] : -1;
-                gv[u] = i < n_entries ? c.gates[t0 * c.k + i] : 0.f;
+    // Stable ranking of the block's entries in (token, slot) order, up to 1024 per round: each warp
+    // ranks its 32 consecutive entries among equal experts (match), writes its per-expert counts,
+    // and one thread per expert turns the warps' counts into bases by an exclusive scan in warp
+    // order, so an entry's row is its expert's next free row + the base + its rank.
+    const int n_entries = nt * c.k;
+    for (int base = 0; base < n_entries; base += 1024) {
+        const int nw = min(32, (n_entries - base + 31) / 32);
+        for (int i = tid; i < nw * c.E; i += blockDim.x) wcnt[i] = 0;
+        __syncthreads();
+        const int i = base + tid;
+        const bool active = warp < nw && i < n_entries;
+        int e = -1, rank = 0;
+        float gv = 0.f;
+        if (warp < nw) {
+            if (active) {
+                e = c.idx[t0 * c.k + i];
+                gv = c.gates[t0 * c.k + i];
+                if (e < 0 || e >= c.E) { set_status(c.status, MOE_STATUS_BOUNDS); e = 0; }
             }
-#pragma unroll
-            for (int u = 0; u < kChunk; ++u) {
-                const int i = base0 + 32 * u + lane;
-                const bool active = i < n_entries;
-                const int flat = t0 * c.k + i;
-                int e = ev[u];
-                if (active && (e < 0 || e >= c.E)) { set_status(c.status, MOE_STATUS_BOUNDS); e = 0; }
-                const unsigned mask = __match_any_sync(0xffffffffu, e);
-                const int rank = __popc(mask & ((1u << lane) - 1u));
-                const int p = active ? nxt[e] + rank : 0;
-                __syncwarp();
-                if (active && lane == __ffs(mask) - 1) nxt[e] += __popc(mask);
-                __syncwarp();
-                if (active) {
-                    if (p < 0 || p >= c.rows_cap) {
-                        set_status(c.status, MOE_STATUS_BOUNDS);
-                    } else {
-                        c.perm[p] = flat;
-                        c.row_token[p] = flat / c.k;
-                        c.row_gate[p] = gv[u];
-                    }
-                }
+            const unsigned mask = __match_any_sync(0xffffffffu, e);
+            rank = __popc(mask & ((1u << lane) - 1u));
+            if (active && lane == __ffs(mask) - 1) wcnt[warp * c.E + e] = __popc(mask);
+        }
+        __syncthreads();
+        if (tid < c.E) {
+            int run = nxt[tid];
+            for (int w = 0; w < nw; ++w) {
+                const int v = wcnt[w * c.E + tid];
+                wcnt[w * c.E + tid] = run;
+                run += v;
+            }
+            nxt[tid] = run;
+        }
+        __syncthreads();
+        if (active) {
+            const int p = wcnt[warp * c.E + e] + rank;
+            const int flat = t0 * c.k + i;
+            if (p < 0 || p >= c.rows_cap) {
+                set_status(c.status, MOE_STATUS_BOUNDS);
+            } else {
+                c.perm[p] = flat;
+                c.row_token[p] = flat / c.k;
+                c.row_gate[p] = gv;
             }
         }
+        __syncthreads();   // the counts are re-zeroed by the next round
     }
-    __syncthreads();
     const int shared_base = off[c.E];
     if (c.has_shared) {
         for (int tt = threadIdx.x; tt < nt; tt += blockDim.x) {
