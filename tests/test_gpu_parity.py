@@ -85,6 +85,23 @@ def test_small_shapes(shape, path):
     layer.close()
 
 
+BIGK = synth.Shape("big_k", T=70, H=256, E=64, k=24, I=128, seed=25)
+
+
+def test_many_experts_per_token():
+    """k = 24: the first 64-token bucketing block holds 1536 routed entries, which the scatter ranks
+    in two rounds of 1024, and the second block is ragged (6 tokens); indices, offsets and the
+    permutation bit-exact, outputs within tolerance (prefill path)."""
+    w = synth.make_layer(BIGK)
+    ol = oracle.OracleLayer.from_shape(w, BIGK)
+    x = gapped_x(BIGK, ol)
+    layer = _layer(w, BIGK, max_tokens=BIGK.T, decode_max_tokens=0)
+    _route_check(layer, ol, x, BIGK)
+    _forward_check(layer, ol, x)
+    _forward_check(layer, ol, x[:65])
+    layer.close()
+
+
 @pytest.mark.parametrize("shape", [TINY, RAGGED], ids=lambda s: s.name)
 def test_poisoned_workspace_changes_no_result(shape):
     """Sanitiser substitute: the workspace starts as 0xFF bytes (NaN / -1) instead of zeros, so a
